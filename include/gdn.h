@@ -1,0 +1,287 @@
+/*
+ * gdn.h -- C ABI of the NVFP4 W4A4 Gated DeltaNet layer forward (sm_100a).
+ *
+ * The method: "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4 W4A4 for
+ * the Recurrent Half of a Hybrid 27B LLM" (franklineh.com research summary)
+ * and "Anthology of the SOTA, theory-128" (section "The account").  A Gated
+ * DeltaNet layer runs every projection, the gate projections included, with
+ * 4-bit NVFP4 weights and activations, and carries a d_k x d_v state per head
+ * through the gated delta rule.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument that names tensor data is a DEVICE pointer owned
+ *     by the caller.  The library never allocates or frees device memory; a
+ *     call that needs scratch space takes a caller-provided workspace whose
+ *     size comes from the matching *_workspace_size query.
+ *   - Every call enqueues its kernels on the caller's stream (a cudaStream_t
+ *     passed as void*; NULL is the legacy default stream) and returns without
+ *     synchronising.  Calls hold no state between them, so calls on different
+ *     streams may run concurrently as long as their buffers do not overlap.
+ *   - Every call returns a gdn_status_t.  Argument checks run on the host
+ *     before anything is launched; on a check failure nothing is enqueued.
+ *     GDN_ERR_CUDA means a launch failed (gdn_last_error() has the CUDA text).
+ *     Device-side waits are bounded: a wait that runs out records
+ *     GDN_ERR_TIMEOUT in a device status word that gdn_stream_check() reads.
+ *   - bf16 is IEEE bfloat16 storage (uint16 bit patterns).
+ *
+ * NVFP4 storage produced by gdn_quantize_nvfp4 and consumed by gdn_gemm_nvfp4
+ *   codes   uint8 [rows, K/2], row-major, row stride K/2 bytes.  Element 2j of
+ *           a row is the low nibble of byte j, element 2j+1 the high nibble.
+ *           A nibble is E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0
+ *           mantissa; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6.
+ *   scales  one E4M3 (bias 7, finite max 448) byte per 16 consecutive
+ *           elements of a row.  Two layouts:
+ *             GDN_SF_LINEAR  [rows, K/16] row-major;
+ *             GDN_SF_TILED   the tensor-core layout: blocks of 128 rows x 64
+ *               elements (4 scales) are 512 contiguous bytes, blocks ordered
+ *               row-block major then K-block; the scale of (row r, element
+ *               group j) sits at byte
+ *                 (r/128)*(K/64)*512 + (j/4)*512 + (r%32)*16 + ((r%128)/32)*4 + j%4.
+ *               The buffer holds ceil(rows/128)*128 rows; bytes of padding
+ *               rows are never read for any stored output.
+ *   g       one FP32 per-tensor DECODE scale: x ~= e2m1 * e4m3 * g.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum      */
+  GDN_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside what the kernels support    */
+  GDN_ERR_ALIGNMENT = 3,         /* a pointer or stride breaks an alignment rule */
+  GDN_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed         */
+  GDN_ERR_TIMEOUT = 5,           /* a bounded device-side wait ran out          */
+  GDN_ERR_WORKSPACE = 6          /* workspace missing or smaller than required  */
+} gdn_status_t;
+
+typedef void* gdn_stream_t; /* cudaStream_t */
+
+/* Text for a status code (static storage). */
+const char* gdn_status_string(int status);
+/* Text of the last CUDA error seen by this thread's calls (static storage). */
+const char* gdn_last_error(void);
+/* Library version, e.g. "0.1.0". */
+const char* gdn_version(void);
+/* Synchronise `stream`, then return and clear the device status word
+ * (GDN_OK, or GDN_ERR_TIMEOUT when a bounded device wait ran out), or
+ * GDN_ERR_CUDA when the synchronisation itself failed. */
+int gdn_stream_check(gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * Step 1: quantize activations to NVFP4.
+ *
+ * Passage: "Why Gated DeltaNet Survives 4-Bit Quantization", section "Why the
+ * 'Fragile' Recurrence is Actually Robust" -- NVFP4 block scaling over groups
+ * of 16 elements, which keeps an outlier's error inside its own block.
+ *
+ * Recipe (FP32, round-to-nearest-even, one operation at a time):
+ *   DYNAMIC mode:      amax_t = max|x| over the tensor,
+ *                      g_enc  = 2688 / amax_t (1 if amax_t == 0; FLT_MAX if
+ *                      the quotient overflows);
+ *   GIVEN_SCALE mode:  g_enc  = *g_enc_in (device scalar, > 0, finite).
+ *   per 16-block:      s = E4M3_satfinite((amax_b / 6) * g_enc);
+ *                      code_i = E2M1_satfinite(x_i * (g_enc / s))
+ *                      (all codes 0 when s == 0; a negative value that rounds
+ *                      to zero keeps its sign bit, code 0x8);
+ *   *g_out = 1 / g_enc (the decode scale).
+ *
+ * x        [rows, cols], element (r, c) at x[r*ld_x + c]; x_dtype
+ *          GDN_DTYPE_BF16 (activations) or GDN_DTYPE_F32 (e.g. FP32 master
+ *          weights); 16-byte aligned, ld_x * element size % 16 == 0.
+ * cols     multiple of 16 (LINEAR) or of 64 (TILED).
+ * codes    uint8 [rows, cols/2] (row stride cols/2), 8-byte aligned.
+ * scales   LINEAR: uint8 [rows, cols/16].  TILED: the buffer of a larger
+ *          matrix whose rows [sf_row_offset, sf_row_offset + rows) this call
+ *          fills (lets separately scaled projections share one operand);
+ *          sf_row_offset must be 0 for LINEAR.
+ * g_out    device float, written with the decode scale.
+ * ws       DYNAMIC mode only: gdn_quantize_workspace_size() bytes, 16-byte
+ *          aligned (holds the running amax; overwritten).  May be NULL in
+ *          GIVEN_SCALE mode.
+ * rows == 0 is valid (only *g_out is written).
+ * ------------------------------------------------------------------------ */
+enum { GDN_QUANT_DYNAMIC = 0, GDN_QUANT_GIVEN_SCALE = 1 };
+enum { GDN_DTYPE_BF16 = 0, GDN_DTYPE_F32 = 1 };
+enum { GDN_SF_TILED = 0, GDN_SF_LINEAR = 1 };
+
+size_t gdn_quantize_workspace_size(void);
+/* Bytes of a TILED scale buffer for a [rows, cols] matrix. */
+size_t gdn_scales_tiled_bytes(int64_t rows, int64_t cols);
+
+int gdn_quantize_nvfp4(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                       int mode, const float* g_enc_in,
+                       uint8_t* codes, uint8_t* scales, int sf_layout,
+                       int64_t sf_row_offset, float* g_out,
+                       void* ws, size_t ws_bytes, gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * Step 2: block-scaled FP4 GEMM  Y[m, n] = sum_k A_hat[m, k] * B_hat[n, k].
+ *
+ * Passage: "Why Gated DeltaNet Survives 4-Bit Quantization", section
+ * "Performance and Efficiency Gains" -- all 496 linear layers, gate
+ * projections included, run with NVFP4 weights and activations; section
+ * "Critical Lessons for Model Serving" -- fusing modules that were scaled
+ * separately mixes up their global scales and silently corrupts the gates,
+ * so every column segment of a fused projection carries its own B scale.
+ *
+ * A   [M, K] NVFP4 (codes + TILED scales), decode scale *g_a (device).
+ * B   [N, K] NVFP4 (codes + TILED scales); segment s covers rows
+ *     [n_begin, n_end) of B and uses decode scale *segs[s].g_b.
+ * The FP32 accumulator of column n in segment s is multiplied by
+ * (*g_a) * (*g_b) and then:
+ *   GDN_EPI_STORE_BF16  out[m*ld_out + (n - n_begin)] = bf16_rne(y)
+ *   GDN_EPI_STORE_F32   out[m*ld_out + (n - n_begin)] = y
+ *   GDN_EPI_LOG_ALPHA   out[...] = -exp(A_log[j]) * softplus(y + dt_bias[j]),
+ *                       j = n - n_begin (FP32; the decay gate of step 3)
+ *   GDN_EPI_BETA        out[...] = sigmoid(y) (FP32; the write strength)
+ * Segments must be sorted, disjoint and cover [0, N); at most
+ * GDN_MAX_SEGMENTS.  Outputs of different segments may share a buffer.
+ *
+ * Shapes: K % 64 == 0, K >= 64; M, N >= 0 arbitrary (ragged tiles handled).
+ * Alignment: codes and scales 16-byte aligned; bf16 outputs 4-byte aligned.
+ * ------------------------------------------------------------------------ */
+enum {
+  GDN_EPI_STORE_BF16 = 0,
+  GDN_EPI_STORE_F32 = 1,
+  GDN_EPI_LOG_ALPHA = 2,
+  GDN_EPI_BETA = 3
+};
+#define GDN_MAX_SEGMENTS 8
+
+typedef struct {
+  const uint8_t* codes;  /* [rows, K/2] */
+  const uint8_t* scales; /* TILED layout */
+} gdn_nvfp4_t;
+
+typedef struct {
+  int64_t n_begin, n_end;
+  int kind;
+  const float* g_b;      /* device scalar: decode scale of these B rows */
+  void* out;
+  int64_t ld_out;        /* elements */
+  const float* A_log;    /* LOG_ALPHA only: [n_end - n_begin] */
+  const float* dt_bias;  /* LOG_ALPHA only: [n_end - n_begin] */
+} gdn_epilogue_segment_t;
+
+int gdn_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B,
+                   int64_t M, int64_t N, int64_t K,
+                   const gdn_epilogue_segment_t* segs, int n_segs,
+                   gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * Step 3: gates, standalone.
+ *
+ * Passage: "Anthology of the SOTA, theory-128", section "The account" -- the
+ * decay is exp(-exp(A) * softplus(a + dt_bias)) and the write strength is a
+ * sigmoid.  (The page prints "softplus(a + b)"; the b there is the per-head
+ * bias dt_bias.)
+ *
+ * a, b            FP32 [M, H] row-major (gate pre-activations).
+ * A_log, dt_bias  FP32 [H].
+ * log_alpha       FP32 [M, H] out: -exp(A_log[h]) * softplus(a + dt_bias[h]).
+ * beta            FP32 [M, H] out: 1 / (1 + exp(-b)).
+ * FP32 with CUDA's expf / log1pf (not the fast intrinsics).
+ * ------------------------------------------------------------------------ */
+int gdn_gates(const float* a, const float* b, int64_t M, int H,
+              const float* A_log, const float* dt_bias,
+              float* log_alpha, float* beta, gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * Step 4: gated delta rule forward (chunked; chunk length 64).
+ *
+ * Passage: "Anthology of the SOTA, theory-128", section "The account" --
+ *   S_t = alpha_t S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T,  o_t = S_t^T q_t,
+ * with q, k L2-normalised per (token, head) over d_k when
+ * GDN_DR_L2NORM_QK is set: x_hat = x / sqrt(||x||^2 + 1e-6).
+ *
+ * q, k   bf16, element (b, t, h, i) at q[(b*T + t)*ld_q + h*dk + i]
+ *        (ld_k likewise); v bf16 with ld_v and dv.  16-byte aligned,
+ *        ld % 8 == 0.
+ * log_alpha, beta  FP32 [B, T, H] contiguous.
+ * S0     FP32 [B, H, dk, dv] initial state, or NULL for zeros.
+ * o      [B, T, H, dv] contiguous; bf16, or FP32 with GDN_DR_O_FP32.
+ * S_T    FP32 [B, H, dk, dv] final state, or NULL.
+ * Supported: dk and dv in {32, 64, 128}; any T >= 0 (a ragged last chunk is
+ * handled); B*H >= 1.  Values of v and of the state must stay inside the
+ * FP16 range (|x| < 65504): the chunk contractions run on FP16 tensor-core
+ * operands with FP32 accumulation.
+ * ws     gdn_delta_rule_workspace_size(...) bytes (may be 0 / NULL).
+ * ------------------------------------------------------------------------ */
+enum { GDN_DR_L2NORM_QK = 1, GDN_DR_O_FP32 = 2 };
+
+size_t gdn_delta_rule_workspace_size(int64_t B, int64_t T, int H, int dk, int dv);
+
+int gdn_delta_rule_fwd(const void* q, const void* k, const void* v,
+                       int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                       const float* log_alpha, const float* beta,
+                       const float* S0, int64_t B, int64_t T, int H, int dk, int dv,
+                       int flags, void* o, float* S_T,
+                       void* ws, size_t ws_bytes, gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * The layer: steps 1-4 and the output projection, in one call.
+ *
+ *   xq = quant(x); [q|k|v|a|b] = gemm(xq, W_qkvab) with gates in the epilogue;
+ *   o  = delta_rule(q, k, v, log_alpha, beta; L2-normalised q, k);
+ *   y  = gemm(quant(o), W_out)  (bf16 out).
+ * No short convolution, output gate, norm or residual.
+ *
+ * Weights are pre-quantized by the caller (gdn_quantize_nvfp4, one call per
+ * projection so each keeps its own decode scale; q, k, v, a, b share one TILED
+ * scale buffer through sf_row_offset).  W_qkvab rows: q [0, H*dk), k [H*dk,
+ * 2*H*dk), v [2*H*dk, 2*H*dk + H*dv), a (H rows), b (H rows); K = d_model.
+ * W_out: [d_model, H*dv].
+ *
+ * x   bf16 [B*T, d_model];  y bf16 [B*T, d_model];  S0 / S_T as in step 4.
+ * ws  gdn_layer_workspace_size(cfg) bytes, 256-byte aligned.  After the call
+ *     it holds the intermediates at the offsets gdn_layer_workspace_offsets
+ *     reports (useful to check each stage).
+ * Supported: d_model % 64 == 0, H*dv % 64 == 0, dk and dv in {32, 64, 128}.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int64_t B, T, d_model;
+  int H, dk, dv;
+} gdn_layer_cfg_t;
+
+typedef struct {
+  gdn_nvfp4_t w_qkvab;   /* [2*H*dk + H*dv + 2*H, d_model] */
+  const float* g_q;      /* device decode scales, one per projection */
+  const float* g_k;
+  const float* g_v;
+  const float* g_a;
+  const float* g_b;
+  gdn_nvfp4_t w_out;     /* [d_model, H*dv] */
+  const float* g_out;
+  const float* A_log;    /* [H] */
+  const float* dt_bias;  /* [H] */
+} gdn_layer_weights_t;
+
+enum {
+  GDN_WS_X_CODES = 0, GDN_WS_X_SCALES, GDN_WS_X_G, GDN_WS_QKV, GDN_WS_LOG_ALPHA,
+  GDN_WS_BETA, GDN_WS_O, GDN_WS_O_CODES, GDN_WS_O_SCALES, GDN_WS_O_G,
+  GDN_WS_QUANT, GDN_WS_SCAN, GDN_WS_COUNT
+};
+
+size_t gdn_layer_workspace_size(const gdn_layer_cfg_t* cfg);
+/* offsets[GDN_WS_COUNT] in bytes from ws: x codes, x scales (TILED), x decode
+ * scale, qkv bf16 [B*T, 2*H*dk + H*dv], log_alpha / beta FP32 [B*T, H],
+ * o bf16 [B*T, H*dv], o codes / scales / decode scale, quantizer and scan
+ * scratch. */
+int gdn_layer_workspace_offsets(const gdn_layer_cfg_t* cfg, int64_t* offsets);
+
+int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg,
+                  const void* x, void* y, const float* S0, float* S_T,
+                  void* ws, size_t ws_bytes, gdn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,206 @@
+// C-ABI entry points: argument checks, workspace arithmetic, status plumbing.
+// Every check runs on the host before anything is enqueued.
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+
+namespace {
+__device__ int g_status_word = GDN_OK;
+
+thread_local char t_last_error[256] = "no error";
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+}  // namespace
+
+int record_cuda_error(cudaError_t err) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(err), cudaGetErrorString(err));
+  return GDN_ERR_CUDA;
+}
+
+int* device_status_word() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_status_ptr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[d] = static_cast<int*>(p);
+  }
+  return g_status_ptr[d];
+}
+
+int num_sms() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_num_sms[d]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    g_num_sms[d] = n;
+  }
+  return g_num_sms[d];
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+namespace {
+constexpr size_t kQuantWs = 256;
+
+cudaStream_t as_stream(gdn_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int check_quant_args(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode, const float* g_enc_in,
+                     const uint8_t* codes, const uint8_t* scales, int sf_layout, int64_t sf_row_offset,
+                     const float* g_out, const void* ws, size_t ws_bytes) {
+  if (rows < 0 || cols <= 0 || ld_x < cols || !g_out) return GDN_ERR_INVALID_ARG;
+  if (x_dtype != GDN_DTYPE_BF16 && x_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARG;
+  const int64_t per16 = x_dtype == GDN_DTYPE_F32 ? 4 : 8;  // elements per 16 bytes
+  if (mode != GDN_QUANT_DYNAMIC && mode != GDN_QUANT_GIVEN_SCALE) return GDN_ERR_INVALID_ARG;
+  if (sf_layout != GDN_SF_TILED && sf_layout != GDN_SF_LINEAR) return GDN_ERR_INVALID_ARG;
+  if (sf_row_offset < 0 || (sf_layout == GDN_SF_LINEAR && sf_row_offset != 0)) return GDN_ERR_INVALID_ARG;
+  if (mode == GDN_QUANT_GIVEN_SCALE && !g_enc_in) return GDN_ERR_INVALID_ARG;
+  if (mode == GDN_QUANT_DYNAMIC && (!ws || ws_bytes < kQuantWs)) return GDN_ERR_WORKSPACE;
+  if (cols % 16 != 0 || (sf_layout == GDN_SF_TILED && cols % 64 != 0)) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (rows > 0 && (!x || !codes || !scales)) return GDN_ERR_INVALID_ARG;
+  if (rows > 0 && (!aligned(x, 16) || ld_x % per16 != 0 || !aligned(codes, 8))) return GDN_ERR_ALIGNMENT;
+  if (ws && !aligned(ws, 16)) return GDN_ERR_ALIGNMENT;
+  if (!aligned(g_out, 4) || (g_enc_in && !aligned(g_enc_in, 4))) return GDN_ERR_ALIGNMENT;
+  return GDN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(int status) {
+  switch (status) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_INVALID_ARG: return "invalid argument";
+    case GDN_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case GDN_ERR_ALIGNMENT: return "pointer or stride alignment";
+    case GDN_ERR_CUDA: return "CUDA error";
+    case GDN_ERR_TIMEOUT: return "device-side wait timed out";
+    case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* gdn_last_error(void) { return t_last_error; }
+
+const char* gdn_version(void) { return "0.1.0"; }
+
+int gdn_stream_check(gdn_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return record_cuda_error(e);
+  int* p = device_status_word();
+  if (!p) return record_cuda_error(cudaErrorInvalidDevice);
+  int word = GDN_OK;
+  e = cudaMemcpy(&word, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  if (word != GDN_OK) {
+    const int zero = GDN_OK;
+    e = cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return record_cuda_error(e);
+  }
+  return word;
+}
+
+size_t gdn_quantize_workspace_size(void) { return kQuantWs; }
+
+size_t gdn_scales_tiled_bytes(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0) return 0;
+  return (size_t)(cdiv(rows, 128) * 128) * (size_t)(cdiv(cols, 64) * 4);
+}
+
+int gdn_quantize_nvfp4(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode,
+                       const float* g_enc_in, uint8_t* codes, uint8_t* scales, int sf_layout, int64_t sf_row_offset,
+                       float* g_out, void* ws, size_t ws_bytes, gdn_stream_t stream) {
+  int st = check_quant_args(x, x_dtype, rows, cols, ld_x, mode, g_enc_in, codes, scales, sf_layout, sf_row_offset, g_out, ws,
+                            ws_bytes);
+  if (st) return st;
+  return launch_quantize(x, x_dtype, rows, cols, ld_x, mode, g_enc_in, codes, scales,
+                         sf_layout == GDN_SF_TILED ? 1 : 0, sf_row_offset, g_out, static_cast<unsigned*>(ws),
+                         as_stream(stream));
+}
+
+int gdn_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B, int64_t M, int64_t N, int64_t K,
+                   const gdn_epilogue_segment_t* segs, int n_segs, gdn_stream_t stream) {
+  if (!A || !B || !g_a || !segs) return GDN_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K <= 0) return GDN_ERR_INVALID_ARG;
+  if (n_segs < 1 || n_segs > GDN_MAX_SEGMENTS) return GDN_ERR_INVALID_ARG;
+  if (K % 64 != 0) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 24)) return GDN_ERR_UNSUPPORTED_SHAPE;
+  int64_t expect = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    const gdn_epilogue_segment_t& s = segs[i];
+    if (s.n_begin != expect || s.n_end <= s.n_begin || !s.g_b || !s.out || s.ld_out <= 0) return GDN_ERR_INVALID_ARG;
+    if (s.kind < GDN_EPI_STORE_BF16 || s.kind > GDN_EPI_BETA) return GDN_ERR_INVALID_ARG;
+    if (s.kind == GDN_EPI_LOG_ALPHA && (!s.A_log || !s.dt_bias)) return GDN_ERR_INVALID_ARG;
+    if (s.ld_out < s.n_end - s.n_begin) return GDN_ERR_INVALID_ARG;
+    if (!aligned(s.out, s.kind == GDN_EPI_STORE_BF16 ? 2 : 4)) return GDN_ERR_ALIGNMENT;
+    expect = s.n_end;
+  }
+  if (expect != N) return GDN_ERR_INVALID_ARG;
+  if (M > 0 && N > 0) {
+    if (!A->codes || !A->scales || !B->codes || !B->scales) return GDN_ERR_INVALID_ARG;
+    if (!aligned(A->codes, 16) || !aligned(B->codes, 16) || !aligned(A->scales, 16) || !aligned(B->scales, 16))
+      return GDN_ERR_ALIGNMENT;
+  }
+  return launch_gemm_nvfp4(A, g_a, B, M, N, K, segs, n_segs, as_stream(stream));
+}
+
+int gdn_gates(const float* a, const float* b, int64_t M, int H, const float* A_log, const float* dt_bias,
+              float* log_alpha, float* beta, gdn_stream_t stream) {
+  if (M < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+  if (M > 0 && (!a || !b || !A_log || !dt_bias || !log_alpha || !beta)) return GDN_ERR_INVALID_ARG;
+  return launch_gates(a, b, M, H, A_log, dt_bias, log_alpha, beta, as_stream(stream));
+}
+
+size_t gdn_delta_rule_workspace_size(int64_t B, int64_t T, int H, int dk, int dv) {
+  (void)B;
+  (void)T;
+  (void)H;
+  (void)dk;
+  (void)dv;
+  return 0;
+}
+
+int gdn_delta_rule_fwd(const void* q, const void* k, const void* v, int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                       const float* log_alpha, const float* beta, const float* S0, int64_t B, int64_t T, int H, int dk,
+                       int dv, int flags, void* o, float* S_T, void* ws, size_t ws_bytes, gdn_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (B < 0 || T < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+  if (flags & ~(GDN_DR_L2NORM_QK | GDN_DR_O_FP32)) return GDN_ERR_INVALID_ARG;
+  if ((dk != 32 && dk != 64 && dk != 128) || (dv != 32 && dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (B * (int64_t)H > (1 << 30) || T > (int64_t)1 << 40) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (ld_q < (int64_t)H * dk || ld_k < (int64_t)H * dk || ld_v < (int64_t)H * dv) return GDN_ERR_INVALID_ARG;
+  if (B > 0 && T > 0) {
+    if (!q || !k || !v || !log_alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || ld_q % 8 || ld_k % 8 || ld_v % 8)
+      return GDN_ERR_ALIGNMENT;
+    if (!aligned(o, (flags & GDN_DR_O_FP32) ? 8 : 4) || !aligned(log_alpha, 4) || !aligned(beta, 4))
+      return GDN_ERR_ALIGNMENT;
+  }
+  if ((S0 && !aligned(S0, 4)) || (S_T && !aligned(S_T, 4))) return GDN_ERR_ALIGNMENT;
+  return launch_delta_rule(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                           static_cast<const uint16_t*>(v), ld_q, ld_k, ld_v, log_alpha, beta, S0, B, T, H, dk, dv,
+                           flags, o, S_T, as_stream(stream));
+}
+
+}  // extern "C"

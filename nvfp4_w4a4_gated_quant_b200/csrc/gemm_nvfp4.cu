@@ -1,0 +1,387 @@
+// Block-scaled NVFP4 GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// Y[m, n] = g_a * g_b(seg(n)) * sum_k e2m1(A[m,k]) sa[m,k/16] e2m1(B[n,k]) sb[n,k/16]
+//
+// Method: every projection of the W4A4 Gated DeltaNet layer, gate projections
+// included ("Why Gated DeltaNet Survives 4-Bit Quantization", section
+// "Performance and Efficiency Gains"), with one decode scale per fused column
+// segment (section "Critical Lessons for Model Serving": modules scaled
+// separately must not share one global scale inside a fused kernel).
+//
+// Design (one CTA per SM, persistent over 128 x 256 output tiles, M fastest):
+//   warp 0        TMA producer: A tile 128 x 256 fp4 and B tile 256 x 256 fp4
+//                 (128-byte rows, 128B swizzle) plus their E4M3 scale blocks
+//                 (untiled bulk copies of the tensor-core scale layout) into a
+//                 4-stage shared-memory ring.  No multicast.
+//   warp 1        TMEM owner and MMA issuer: copies each stage's scales to
+//                 TMEM (tcgen05.cp 32x128b.warpx4), then issues
+//                 tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128,
+//                 N=256, K=64) into a 128 x 256 FP32 accumulator in TMEM;
+//                 tcgen05.commit frees the stage / publishes the tile.
+//   warps 4..11   epilogue: tcgen05.ld of 32-column slices, the per-segment
+//                 scale, then bf16 / FP32 stores or the gate functions.
+// Every mbarrier wait is bounded; a wait that runs out records
+// GDN_ERR_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "gate_math.cuh"
+#include "kernels.h"
+
+namespace gdn {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 256;                 // fp4 elements per stage (128 bytes per row)
+constexpr int KSTEP = 64;               // K of one MMA
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK / 2;    // 16 KiB
+constexpr int B_BYTES = BN * BK / 2;    // 32 KiB
+constexpr int SFA_BYTES = (BK / KSTEP) * 512;          // 2 KiB
+constexpr int SFB_BYTES = (BN / 128) * (BK / KSTEP) * 512;  // 4 KiB
+constexpr int NUM_THREADS = 384;
+constexpr int EPI_WARP0 = 4;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;         // 256 FP32 columns
+constexpr uint32_t SFA_COL = 256;       // 4 k-steps x 4 columns
+constexpr uint32_t SFB_COL = 272;       // 4 k-steps x 8 columns
+
+constexpr size_t SMEM_BYTES =
+    1024 /*alignment slack*/ + (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 256;
+
+struct Segment {
+  int n_begin, n_end, kind;
+  const float* g_b;
+  void* out;
+  int64_t ld_out;
+  const float* A_log;
+  const float* dt_bias;
+};
+
+struct Params {
+  int M, N, K;
+  int num_m, num_n, num_tiles;
+  int kc;                      // K / 64: scale blocks per 128-row block
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* g_a;
+  int n_segs;
+  Segment segs[GDN_MAX_SEGMENTS];
+  int* status;
+};
+
+// K-major operand in 128-byte swizzled rows, 8-row core groups 1024 B apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                 // leading byte offset (unused when swizzled)
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset
+  d |= (uint64_t)1 << 46;                 // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                 // 128-byte swizzle
+  return d;
+}
+// Scale block for tcgen05.cp: 32 rows of 16 bytes, 8-row groups 128 B apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+// Instruction descriptor: E2M1 x E2M1, UE4M3 scales, FP32 accumulate,
+// both operands K-major, M = 128, N = 256, dense, K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (i > 64) __nanosleep(32);
+  }
+  report_status(status, GDN_ERR_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ int find_segment(const Params& p, int n) {
+  int s = 0;
+#pragma unroll 1
+  while (s + 1 < p.n_segs && n >= p.segs[s].n_end) ++s;
+  return s;
+}
+
+__device__ __forceinline__ void epilogue_store_one(const Segment& sg, int m, int n, float y) {
+  const int64_t off = (int64_t)m * sg.ld_out + (n - sg.n_begin);
+  switch (sg.kind) {
+    case GDN_EPI_STORE_BF16:
+      reinterpret_cast<uint16_t*>(sg.out)[off] = (uint16_t)f32_to_bf16_bits(y);
+      break;
+    case GDN_EPI_STORE_F32:
+      reinterpret_cast<float*>(sg.out)[off] = y;
+      break;
+    case GDN_EPI_LOG_ALPHA: {
+      const int j = n - sg.n_begin;
+      reinterpret_cast<float*>(sg.out)[off] = gate_log_alpha(y, sg.A_log[j], sg.dt_bias[j]);
+      break;
+    }
+    default:
+      reinterpret_cast<float*>(sg.out)[off] = gate_beta(y);
+      break;
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                  const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sSFA = sB + STAGES * B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, NUM_EPI_WARPS);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_ptr, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+
+  const int num_kb = (p.K + BK - 1) / BK;
+  const int ksteps_total = p.K / KSTEP;
+  const int sf_blocks_n = (p.N + 127) / 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------- producer
+      uint32_t it = 0;
+      uint32_t last_round[STAGES];
+      bool issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = false, last_round[s] = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+        const int mb = tile % p.num_m, nb = tile / p.num_m;
+        const int nh = min(2, sf_blocks_n - 2 * nb);
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t round = it / STAGES;
+          if (!wait_or_abort(&empty[s], (round & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
+          const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
+          const uint32_t bytes = A_BYTES + B_BYTES + (uint32_t)nks * 512u * (1u + (uint32_t)nh);
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], kb * (BK / 2), mb * BM);
+          tma_load_2d(sB + s * B_BYTES, &tmap_b, &full[s], kb * (BK / 2), nb * BN);
+          bulk_load(sSFA + s * SFA_BYTES, p.sfa + ((int64_t)mb * p.kc + kb * 4) * 512, nks * 512, &full[s]);
+          for (int h = 0; h < nh; ++h)
+            bulk_load(sSFB + s * SFB_BYTES + h * 2048, p.sfb + ((int64_t)(2 * nb + h) * p.kc + kb * 4) * 512,
+                      nks * 512, &full[s]);
+          issued[s] = true;
+          last_round[s] = round;
+        }
+      }
+      // Drain: every copy this thread issued lands before the CTA exits.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s]) {
+          for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&full[s], last_round[s] & 1); ++i) __nanosleep(32);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      uint32_t it = 0, tile_iter = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
+        const int nb = tile / p.num_m;
+        const int nh = min(2, sf_blocks_n - 2 * nb);
+        if (!wait_or_abort(acc_empty, (tile_iter & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t round = it / STAGES;
+          if (!wait_or_abort(&full[s], round & 1, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
+          const uint32_t sfa_s = smem_u32(sSFA + s * SFA_BYTES);
+          const uint32_t sfb_s = smem_u32(sSFB + s * SFB_BYTES);
+          for (int j = 0; j < nks; ++j) {
+            tc_cp_32x128b_warpx4(tmem + SFA_COL + j * 4, desc_sf(sfa_s + j * 512));
+            for (int h = 0; h < nh; ++h)
+              tc_cp_32x128b_warpx4(tmem + SFB_COL + j * 8 + h * 4, desc_sf(sfb_s + (h * 4 + j) * 512));
+          }
+          const uint32_t a_s = smem_u32(sA + s * A_BYTES);
+          const uint32_t b_s = smem_u32(sB + s * B_BYTES);
+          for (int j = 0; j < nks; ++j)
+            tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc,
+                        tmem + SFA_COL + j * 4, tmem + SFB_COL + j * 8, (kb > 0 || j > 0) ? 1u : 0u);
+          tc_commit(&empty[s]);
+        }
+        if (ok) tc_commit(acc_full);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= EPI_WARP0) {
+    // --------------------------------------------------------- epilogue
+    const int ew = warp - EPI_WARP0;
+    const int quad = warp & 3;            // TMEM lanes quad*32 .. quad*32+31
+    const int half = ew >> 2;             // columns half*128 .. half*128+127
+    uint32_t tile_iter = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
+      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      bool ok = true;
+      if (lane == 0) ok = wait_or_abort(acc_full, tile_iter & 1, p.status, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const int m = mb * BM + quad * 32 + lane;
+      const float g_a = *p.g_a;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        const int col0 = half * 128 + c * 32;
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + col0, r);
+        tc_wait_ld();
+        if (c == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+        }
+        const int n0 = nb * BN + col0;
+        if (m >= p.M || n0 >= p.N) continue;
+        const int s0 = find_segment(p, n0);
+        const Segment& sg = p.segs[s0];
+        const bool whole = (n0 + 31 < sg.n_end) && (n0 + 31 < p.N);
+        const int64_t off = (int64_t)m * sg.ld_out + (n0 - sg.n_begin);
+        if (whole && sg.kind == GDN_EPI_STORE_BF16 && ((reinterpret_cast<uintptr_t>(sg.out) + off * 2) % 16) == 0) {
+          const float alpha = __fmul_rn(g_a, *sg.g_b);
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(sg.out) + off);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float y0 = __fmul_rn(__uint_as_float(r[v * 8 + 2 * e]), alpha);
+              const float y1 = __fmul_rn(__uint_as_float(r[v * 8 + 2 * e + 1]), alpha);
+              w[e] = f32_to_bf16_bits(y0) | (f32_to_bf16_bits(y1) << 16);
+            }
+            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+#pragma unroll 1
+          for (int i = 0; i < 32; ++i) {
+            const int n = n0 + i;
+            if (n >= p.N) break;
+            const Segment& sgi = p.segs[find_segment(p, n)];
+            const float y = __fmul_rn(__uint_as_float(r[i]), __fmul_rn(g_a, *sgi.g_b));
+            epilogue_store_one(sgi, m, n, y);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+int make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, uint32_t box_rows) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return record_cuda_error(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  cuuint32_t box[2] = {(cuuint32_t)(BK / 2), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return record_cuda_error(cudaErrorInvalidValue);
+  return GDN_OK;
+}
+
+}  // namespace
+
+int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B, int64_t M, int64_t N, int64_t K,
+                      const gdn_epilogue_segment_t* segs, int n_segs, cudaStream_t stream) {
+  if (M == 0 || N == 0) return GDN_OK;
+  Params p{};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.num_m = (int)cdiv(M, BM);
+  p.num_n = (int)cdiv(N, BN);
+  p.num_tiles = p.num_m * p.num_n;
+  p.kc = (int)(K / 64);
+  p.sfa = A->scales;
+  p.sfb = B->scales;
+  p.g_a = g_a;
+  p.n_segs = n_segs;
+  for (int i = 0; i < n_segs; ++i) {
+    p.segs[i].n_begin = (int)segs[i].n_begin;
+    p.segs[i].n_end = (int)segs[i].n_end;
+    p.segs[i].kind = segs[i].kind;
+    p.segs[i].g_b = segs[i].g_b;
+    p.segs[i].out = segs[i].out;
+    p.segs[i].ld_out = segs[i].ld_out;
+    p.segs[i].A_log = segs[i].A_log;
+    p.segs[i].dt_bias = segs[i].dt_bias;
+  }
+  p.status = device_status_word();
+  CUtensorMap ta, tb;
+  int st = make_codes_map(&ta, A->codes, M, K, BM);
+  if (st) return st;
+  st = make_codes_map(&tb, B->codes, N, K, BN);
+  if (st) return st;
+  cudaError_t attr_err =
+      cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (attr_err != cudaSuccess) return record_cuda_error(attr_err);
+  const int grid = (int)std::min<int64_t>(p.num_tiles, num_sms());
+  gemm_nvfp4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ta, tb, p);
+  return check_launch();
+}
+
+}  // namespace gdn

@@ -1,0 +1,26 @@
+// Internal launchers of the sm_100a kernels (host side, no validation: the
+// C-ABI entry points in api.cu check every argument before calling these).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+int launch_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, int mode, const float* g_enc_in,
+                    uint8_t* codes, uint8_t* scales, int tiled, int64_t row_off, float* g_out, unsigned* amax_ws,
+                    cudaStream_t stream);
+
+int launch_gates(const float* a, const float* b, int64_t M, int H, const float* A_log, const float* dt_bias,
+                 float* log_alpha, float* beta, cudaStream_t stream);
+
+int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B, int64_t M, int64_t N,
+                      int64_t K, const gdn_epilogue_segment_t* segs, int n_segs, cudaStream_t stream);
+
+int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
+                      int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
+                      int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, cudaStream_t stream);
+
+}  // namespace gdn

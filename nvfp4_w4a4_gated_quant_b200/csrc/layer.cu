@@ -1,0 +1,126 @@
+// The W4A4 Gated DeltaNet layer forward: quantize -> fused q/k/v/a/b GEMM with
+// the gates in its epilogue -> chunked delta rule -> quantize -> output GEMM.
+// Five kernel launches (plus one 4-byte memset per quantization) on the
+// caller's stream; every intermediate lives in the caller's workspace.
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace gdn;
+
+namespace {
+
+int64_t align256(int64_t x) { return (x + 255) & ~(int64_t)255; }
+
+bool cfg_ok(const gdn_layer_cfg_t* c) {
+  return c && c->B >= 0 && c->T >= 0 && c->d_model > 0 && c->H > 0 && c->dk > 0 && c->dv > 0;
+}
+
+int layout(const gdn_layer_cfg_t* c, int64_t* off, int64_t* total) {
+  const int64_t M = c->B * c->T;
+  const int64_t D = c->d_model;
+  const int64_t HV = (int64_t)c->H * c->dv;
+  const int64_t NQKV = 2 * (int64_t)c->H * c->dk + HV;
+  int64_t sizes[GDN_WS_COUNT];
+  sizes[GDN_WS_X_CODES] = M * D / 2;
+  sizes[GDN_WS_X_SCALES] = (int64_t)gdn_scales_tiled_bytes(M, D);
+  sizes[GDN_WS_X_G] = 4;
+  sizes[GDN_WS_QKV] = M * NQKV * 2;
+  sizes[GDN_WS_LOG_ALPHA] = M * c->H * 4;
+  sizes[GDN_WS_BETA] = M * c->H * 4;
+  sizes[GDN_WS_O] = M * HV * 2;
+  sizes[GDN_WS_O_CODES] = M * HV / 2;
+  sizes[GDN_WS_O_SCALES] = (int64_t)gdn_scales_tiled_bytes(M, HV);
+  sizes[GDN_WS_O_G] = 4;
+  sizes[GDN_WS_QUANT] = (int64_t)gdn_quantize_workspace_size();
+  sizes[GDN_WS_SCAN] = (int64_t)gdn_delta_rule_workspace_size(c->B, c->T, c->H, c->dk, c->dv);
+  int64_t pos = 0;
+  for (int i = 0; i < GDN_WS_COUNT; ++i) {
+    off[i] = pos;
+    pos += align256(sizes[i]);
+  }
+  *total = pos;
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_layer_workspace_size(const gdn_layer_cfg_t* cfg) {
+  if (!cfg_ok(cfg)) return 0;
+  int64_t off[GDN_WS_COUNT], total = 0;
+  layout(cfg, off, &total);
+  return (size_t)total;
+}
+
+int gdn_layer_workspace_offsets(const gdn_layer_cfg_t* cfg, int64_t* offsets) {
+  if (!cfg_ok(cfg) || !offsets) return GDN_ERR_INVALID_ARG;
+  int64_t total = 0;
+  return layout(cfg, offsets, &total);
+}
+
+int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, const void* x, void* y, const float* S0,
+                  float* S_T, void* ws, size_t ws_bytes, gdn_stream_t stream) {
+  if (!w || !cfg_ok(cfg)) return GDN_ERR_INVALID_ARG;
+  const int64_t M = cfg->B * cfg->T;
+  const int64_t D = cfg->d_model;
+  const int H = cfg->H, dk = cfg->dk, dv = cfg->dv;
+  const int64_t HK = (int64_t)H * dk, HV = (int64_t)H * dv;
+  const int64_t NQKV = 2 * HK + HV;
+  if (D % 64 != 0 || HV % 64 != 0) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if ((dk != 32 && dk != 64 && dk != 128) || (dv != 32 && dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED_SHAPE;
+  int64_t off[GDN_WS_COUNT], total = 0;
+  layout(cfg, off, &total);
+  if (!ws || (int64_t)ws_bytes < total) return GDN_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return GDN_ERR_ALIGNMENT;
+  if (!w->g_q || !w->g_k || !w->g_v || !w->g_a || !w->g_b || !w->g_out || !w->A_log || !w->dt_bias)
+    return GDN_ERR_INVALID_ARG;
+  if (M > 0) {
+    if (!x || !y || !w->w_qkvab.codes || !w->w_qkvab.scales || !w->w_out.codes || !w->w_out.scales)
+      return GDN_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16)) return GDN_ERR_ALIGNMENT;
+  }
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* x_codes = base + off[GDN_WS_X_CODES];
+  uint8_t* x_scales = base + off[GDN_WS_X_SCALES];
+  float* x_g = reinterpret_cast<float*>(base + off[GDN_WS_X_G]);
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(base + off[GDN_WS_QKV]);
+  float* log_alpha = reinterpret_cast<float*>(base + off[GDN_WS_LOG_ALPHA]);
+  float* beta = reinterpret_cast<float*>(base + off[GDN_WS_BETA]);
+  uint16_t* o = reinterpret_cast<uint16_t*>(base + off[GDN_WS_O]);
+  uint8_t* o_codes = base + off[GDN_WS_O_CODES];
+  uint8_t* o_scales = base + off[GDN_WS_O_SCALES];
+  float* o_g = reinterpret_cast<float*>(base + off[GDN_WS_O_G]);
+  void* qws = base + off[GDN_WS_QUANT];
+  void* sws = base + off[GDN_WS_SCAN];
+  const size_t qws_bytes = gdn_quantize_workspace_size();
+  gdn_stream_t s = stream;
+
+  int st = gdn_quantize_nvfp4(x, GDN_DTYPE_BF16, M, D, D, GDN_QUANT_DYNAMIC, nullptr, x_codes, x_scales, GDN_SF_TILED, 0, x_g, qws,
+                              qws_bytes, s);
+  if (st) return st;
+
+  gdn_nvfp4_t xa{x_codes, x_scales};
+  gdn_epilogue_segment_t seg[5] = {};
+  seg[0] = {0, HK, GDN_EPI_STORE_BF16, w->g_q, qkv, NQKV, nullptr, nullptr};
+  seg[1] = {HK, 2 * HK, GDN_EPI_STORE_BF16, w->g_k, qkv + HK, NQKV, nullptr, nullptr};
+  seg[2] = {2 * HK, NQKV, GDN_EPI_STORE_BF16, w->g_v, qkv + 2 * HK, NQKV, nullptr, nullptr};
+  seg[3] = {NQKV, NQKV + H, GDN_EPI_LOG_ALPHA, w->g_a, log_alpha, H, w->A_log, w->dt_bias};
+  seg[4] = {NQKV + H, NQKV + 2 * H, GDN_EPI_BETA, w->g_b, beta, H, nullptr, nullptr};
+  st = gdn_gemm_nvfp4(&xa, x_g, &w->w_qkvab, M, NQKV + 2 * H, D, seg, 5, s);
+  if (st) return st;
+
+  st = gdn_delta_rule_fwd(qkv, qkv + HK, qkv + 2 * HK, NQKV, NQKV, NQKV, log_alpha, beta, S0, cfg->B, cfg->T, H, dk, dv,
+                          GDN_DR_L2NORM_QK, o, S_T, sws, 0, s);
+  if (st) return st;
+
+  st = gdn_quantize_nvfp4(o, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_DYNAMIC, nullptr, o_codes, o_scales, GDN_SF_TILED, 0, o_g, qws,
+                          qws_bytes, s);
+  if (st) return st;
+
+  gdn_nvfp4_t oa{o_codes, o_scales};
+  gdn_epilogue_segment_t yseg = {0, D, GDN_EPI_STORE_BF16, w->g_out, y, D, nullptr, nullptr};
+  return gdn_gemm_nvfp4(&oa, o_g, &w->w_out, M, D, HV, &yseg, 1, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,208 @@
+// NVFP4 activation quantizer: per-tensor amax, E4M3 block scales, E2M1 codes.
+//
+// Method: "Why Gated DeltaNet Survives 4-Bit Quantization", section "Why the
+// 'Fragile' Recurrence is Actually Robust" -- NVFP4 scales every 16-element
+// block separately.  Two HBM-bound passes:
+//   amax_kernel   max |x| over the tensor (bf16 bit patterns, one atomicMax
+//                 per CTA on the FP32 bits of the result);
+//   quant_kernel  one thread per 16-element block: two 16-byte loads, the
+//                 block scale, eight packed code bytes and one scale byte.
+// The FP32 operation order is fixed (see gdn.h); divisions and products use
+// the round-to-nearest intrinsics so no contraction or approximation changes
+// a code.  E4M3 and E2M1 rounding use the hardware cvt.rn.satfinite forms.
+#include <float.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+namespace {
+
+__device__ __forceinline__ uint4 ld_vec(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// Input element types: bf16 (8 per 16-byte vector) or FP32 (4 per vector).
+struct Bf16In {
+  static constexpr int kPerVec = 8;
+  __device__ static uint32_t absmax_bits(uint4 v) {  // FP32 bits of max |x|
+    uint32_t m = 0;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m = max(m, w[i] & 0x7FFFu);
+      m = max(m, (w[i] >> 16) & 0x7FFFu);
+    }
+    return m << 16;
+  }
+  __device__ static void to_f32(uint4 v, float* out) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      out[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+      out[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+  }
+};
+struct F32In {
+  static constexpr int kPerVec = 4;
+  __device__ static uint32_t absmax_bits(uint4 v) {
+    return max(max(v.x & 0x7FFFFFFFu, v.y & 0x7FFFFFFFu), max(v.z & 0x7FFFFFFFu, v.w & 0x7FFFFFFFu));
+  }
+  __device__ static void to_f32(uint4 v, float* out) {
+    out[0] = __uint_as_float(v.x);
+    out[1] = __uint_as_float(v.y);
+    out[2] = __uint_as_float(v.z);
+    out[3] = __uint_as_float(v.w);
+  }
+};
+
+template <typename In, typename E>
+__global__ void amax_kernel(const E* __restrict__ x, int64_t rows, int64_t vpr, int64_t ld,
+                            unsigned* __restrict__ amax_bits) {
+  uint32_t m = 0;
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    const E* row = x + r * ld;
+    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < vpr; c += (int64_t)gridDim.x * blockDim.x)
+      m = max(m, In::absmax_bits(ld_vec(row + c * In::kPerVec)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ uint32_t red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0 && m) atomicMax(amax_bits, m);  // FP32 bits of |x| order like the values
+  }
+}
+
+__device__ __forceinline__ float encode_scale_from_amax(float amax) {
+  if (amax == 0.0f) return 1.0f;
+  float g = __fdiv_rn(2688.0f, amax);
+  return (g > FLT_MAX) ? FLT_MAX : g;
+}
+
+// E4M3 byte -> FP32 value (exact).
+__device__ __forceinline__ float e4m3_value(uint32_t s) {
+  uint32_t e = (s >> 3) & 15u, m = s & 7u;
+  if (e == 0) return (float)m * 0.001953125f;  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+__device__ __forceinline__ uint32_t e4m3_satfinite(float v) {
+  uint16_t out;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %1;\n\tmov.b16 %0, t;\n\t}"
+      : "=h"(out)
+      : "f"(v));
+  return out & 0xFFu;
+}
+
+// Four pairs -> 4 bytes; element 2j in the low nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8(const float* r) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(r[0]), "f"(r[1]), "f"(r[2]), "f"(r[3]), "f"(r[4]), "f"(r[5]), "f"(r[6]), "f"(r[7]));
+  return out;
+}
+
+template <typename In, typename E>
+__global__ void quant_kernel(const E* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                             int mode, const float* __restrict__ g_enc_in,
+                             const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                             uint8_t* __restrict__ scales, int tiled, int64_t row_off,
+                             float* __restrict__ g_out) {
+  const float g_enc = (mode == GDN_QUANT_DYNAMIC) ? encode_scale_from_amax(__uint_as_float(*amax_bits))
+                                                  : *g_enc_in;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = __fdiv_rn(1.0f, g_enc);
+  const int64_t bpr = cols >> 4;  // 16-element blocks per row
+  const int64_t kc = cols >> 6;   // 64-element scale chunks per row (TILED)
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    const E* row = x + r * ld;
+    for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < bpr; j += (int64_t)gridDim.x * blockDim.x) {
+      constexpr int NV = 16 / In::kPerVec;
+      uint4 vv[NV];
+      uint32_t mb = 0;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        vv[i] = ld_vec(row + j * 16 + i * In::kPerVec);
+        mb = max(mb, In::absmax_bits(vv[i]));
+      }
+      const float amax_b = __uint_as_float(mb);
+      const float s_f = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g_enc);
+      const uint32_t s = e4m3_satfinite(s_f);
+      const float s_val = e4m3_value(s);
+      uint2 packed = make_uint2(0u, 0u);
+      if (s_val > 0.0f) {
+        const float inv = __fdiv_rn(g_enc, s_val);
+        float rr[16];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) In::to_f32(vv[i], rr + i * In::kPerVec);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rr[i] = __fmul_rn(rr[i], inv);
+        packed.x = e2m1x8(rr);
+        packed.y = e2m1x8(rr + 8);
+      }
+      *reinterpret_cast<uint2*>(codes + r * (cols >> 1) + j * 8) = packed;
+      if (tiled) {
+        const int64_t R = r + row_off;
+        const int64_t off = (R >> 7) * kc * 512 + (j >> 2) * 512 + (R & 31) * 16 + ((R & 127) >> 5) * 4 + (j & 3);
+        scales[off] = (uint8_t)s;
+      } else {
+        scales[r * bpr + j] = (uint8_t)s;
+      }
+    }
+  }
+}
+
+void grid_for_rows(int64_t rows, int64_t per_row_items, int threads, dim3& grid) {
+  const int64_t gx = std::min<int64_t>(cdiv(per_row_items, threads), 1024);
+  const int64_t want = (int64_t)num_sms() * 16;  // CTAs in flight
+  int64_t gy = std::max<int64_t>(1, want / std::max<int64_t>(gx, 1));
+  gy = std::min<int64_t>(gy, std::max<int64_t>(rows, 1));
+  gy = std::min<int64_t>(gy, 65535);
+  grid = dim3((unsigned)std::max<int64_t>(gx, 1), (unsigned)gy, 1);
+}
+
+template <typename In, typename E>
+int launch_quantize_t(const E* x, int64_t rows, int64_t cols, int64_t ld, int mode, const float* g_enc_in,
+                    uint8_t* codes, uint8_t* scales, int tiled, int64_t row_off, float* g_out, unsigned* amax_ws,
+                    cudaStream_t stream) {
+  const int threads = 256;
+  if (mode == GDN_QUANT_DYNAMIC) {
+    cudaError_t e = cudaMemsetAsync(amax_ws, 0, sizeof(unsigned), stream);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    if (rows > 0) {
+      dim3 grid;
+      grid_for_rows(rows, cols / In::kPerVec, threads, grid);
+      amax_kernel<In, E><<<grid, threads, 0, stream>>>(x, rows, cols / In::kPerVec, ld, amax_ws);
+      int st = check_launch();
+      if (st) return st;
+    }
+  }
+  dim3 grid;
+  grid_for_rows(rows, cols / 16, threads, grid);
+  quant_kernel<In, E><<<grid, threads, 0, stream>>>(x, rows, cols, ld, mode, g_enc_in, amax_ws, codes, scales, tiled,
+                                             row_off, g_out);
+  return check_launch();
+}
+
+}  // namespace
+
+int launch_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, int mode,
+                    const float* g_enc_in, uint8_t* codes, uint8_t* scales, int tiled, int64_t row_off, float* g_out,
+                    unsigned* amax_ws, cudaStream_t stream) {
+  if (x_dtype == GDN_DTYPE_F32)
+    return launch_quantize_t<F32In>(static_cast<const float*>(x), rows, cols, ld, mode, g_enc_in, codes, scales,
+                                    tiled, row_off, g_out, amax_ws, stream);
+  return launch_quantize_t<Bf16In>(static_cast<const uint16_t*>(x), rows, cols, ld, mode, g_enc_in, codes, scales,
+                                   tiled, row_off, g_out, amax_ws, stream);
+}
+
+}  // namespace gdn

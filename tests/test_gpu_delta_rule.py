@@ -1,0 +1,99 @@
+"""GPU parity of step 4, the chunked gated delta rule, against the FP64 oracle.
+
+"Anthology of the SOTA, theory-128", section "The account":
+S_t = alpha_t S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T, o_t = S_t^T q_t over
+L2-normalised q, k.  Tolerance: 2e-3 relative Frobenius on o (FP32 output) and
+on the final state, the bound the task states for 32K tokens.  Both sides get
+the same bf16 q / k / v and the same FP32 gates.
+"""
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_w4a4_gated_quant_b200 import _lib, inputs
+from oracle.delta_rule import delta_rule_chunked
+from oracle.gates import gates as oracle_gates
+from tests._helpers import bf16_cuda, f32_cuda, rel_fro, to_np
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def _case(B, T, H, dk, dv, seed, with_s0=False):
+    rng = np.random.default_rng(seed)
+    q = inputs.to_bf16_values(rng.standard_normal((B, T, H, dk), dtype=np.float32))
+    k = inputs.to_bf16_values(rng.standard_normal((B, T, H, dk), dtype=np.float32))
+    v = inputs.to_bf16_values(rng.standard_normal((B, T, H, dv), dtype=np.float32))
+    a = rng.standard_normal((B, T, H)).astype(np.float32)
+    b = rng.standard_normal((B, T, H)).astype(np.float32)
+    A = rng.uniform(-2, 1, H)
+    dt = rng.uniform(-1, 1, H)
+    la, be = oracle_gates(a, b, A, dt)
+    la = la.astype(np.float32)
+    be = be.astype(np.float32)
+    S0 = (rng.standard_normal((B, H, dk, dv)) * 0.5).astype(np.float32) if with_s0 else None
+    return q, k, v, la, be, S0
+
+
+def _run(q, k, v, la, be, S0, o_fp32=True):
+    o, S = _lib.gdn_delta_rule_fwd(bf16_cuda(q), bf16_cuda(k), bf16_cuda(v), f32_cuda(la), f32_cuda(be),
+                                   S0=None if S0 is None else f32_cuda(S0), o_fp32=o_fp32)
+    _lib.stream_check()
+    return to_np(o).astype(np.float64), to_np(S).astype(np.float64)
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,seed,s0", [
+    (1, 64, 2, 128, 128, 0, False),     # one full chunk, 4 chains -> 16-column slices
+    (2, 200, 3, 128, 128, 1, True),     # ragged last chunk, initial state
+    (1, 1, 2, 128, 64, 2, False),       # a single token
+    (1, 65, 20, 128, 128, 3, False),    # 20 chains -> 32-column slices
+    (2, 130, 20, 128, 64, 4, True),     # 40 chains, dv 64
+    (2, 96, 40, 128, 128, 5, False),    # 80 chains -> whole 128-column state per CTA
+    (1, 160, 2, 32, 32, 6, True),       # the tiny layer's head dims
+    (1, 100, 3, 64, 64, 7, False),
+])
+def test_delta_rule_matches_oracle(B, T, H, dk, dv, seed, s0):
+    q, k, v, la, be, S0 = _case(B, T, H, dk, dv, seed, s0)
+    o, S = _run(q, k, v, la, be, S0)
+    o_ref, S_ref = delta_rule_chunked(q, k, v, la, be, S0=S0)
+    assert rel_fro(o, o_ref) < TOL, rel_fro(o, o_ref)
+    assert rel_fro(S, S_ref) < TOL, rel_fro(S, S_ref)
+
+
+def test_delta_rule_bf16_output():
+    q, k, v, la, be, S0 = _case(1, 190, 4, 128, 128, 9)
+    o, _ = _run(q, k, v, la, be, S0, o_fp32=False)
+    o_ref, _ = delta_rule_chunked(q, k, v, la, be)
+    # bf16 storage adds its own rounding (~1.5e-3 relative RMS) on top
+    assert rel_fro(o, o_ref) < 3e-3
+
+
+def test_delta_rule_empty_sequence_returns_initial_state():
+    q, k, v, la, be, S0 = _case(1, 0, 2, 128, 128, 10, True)
+    o, S = _run(q, k, v, la, be, S0)
+    np.testing.assert_array_equal(S, S0)
+
+
+def test_delta_rule_segments_with_state_carry():
+    """Two calls over [0, 150) and [150, 300) with the state carried equal
+    one call over [0, 300) (checkpoint / resume of a long prefill)."""
+    q, k, v, la, be, _ = _case(1, 300, 4, 128, 128, 12)
+    o_all, S_all = _run(q, k, v, la, be, None)
+    o1, S1 = _run(q[:, :150], k[:, :150], v[:, :150], la[:, :150], be[:, :150], None)
+    o2, S2 = _run(q[:, 150:], k[:, 150:], v[:, 150:], la[:, 150:], be[:, 150:], S1.astype(np.float32))
+    assert rel_fro(np.concatenate([o1, o2], 1), o_all) < 1e-3
+    assert rel_fro(S2, S_all) < 1e-3
+
+
+def test_delta_rule_scan_workload_32k():
+    """The scan workload: B=1, T=32768, H=16, d=128 (gates from a, b as the
+    layer computes them); o and S_T within 2e-3 of the FP64 oracle."""
+    d = inputs.scan_workload()
+    la, be = oracle_gates(d["a"], d["b"], d["A_log"], d["dt_bias"])
+    la = la.astype(np.float32)
+    be = be.astype(np.float32)
+    o, S = _run(d["q"], d["k"], d["v"], la, be, None)
+    o_ref, S_ref = delta_rule_chunked(d["q"], d["k"], d["v"], la, be)
+    e_o, e_s = rel_fro(o, o_ref), rel_fro(S, S_ref)
+    print(f"scan 32K: rel_fro o {e_o:.3e}  S_T {e_s:.3e}")
+    assert e_o < TOL and e_s < TOL
