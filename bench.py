@@ -1,0 +1,486 @@
+"""Benchmark: W4A4 Gated DeltaNet layer prefill on B200.
+
+One step = one full layer forward (every hot-path stage: quantize x, fused
+q/k/v/a/b NVFP4 GEMM with the gates in its epilogue, chunked delta rule,
+quantize o, output NVFP4 GEMM) over the layer workload: B=4 sequences x
+T=8192 tokens, d_model=5120, H=32 heads of d=128, synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  N > 1 runs one process per GPU (launched by
+torch.distributed.run); every rank runs its own independent batch (weak
+scaling, no data-path collective) and the time is the max over ranks.
+``--impl reference`` times the CPU oracle (the plain FP64 / FP32 restatement
+of the method) on the host cores over a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN W4A4 layer prefill tokens/s"
+UNIT = "tokens/s"
+WORKLOAD = dict(B=4, T=8192, d_model=5120, H=32, dk=128, dv=128)
+WORKLOAD_NAME = "gdn_w4a4_layer_prefill B=4 T=8192 d_model=5120 H=32 dk=dv=128"
+CPU_SAMPLE_T = 256            # tokens of one sequence for the oracle sample
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        p = {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+             "bf16_tflops_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]), "source": "measured"}
+    return p
+
+
+# ------------------------------------------------------------ clock sampler --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s in sm if smax and s > 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- our path --
+def stage_costs(B, T, d_model, H, dk, dv):
+    """Algorithmic bytes (HBM-bound stages) or FLOPs (contractions) of one
+    launch of each stage of the layer."""
+    M = B * T
+    HK, HV = H * dk, H * dv
+    N1 = 2 * HK + HV + 2 * H
+    return {
+        "quant_x": ("hbm", M * d_model * 2 + M * d_model // 2 + M * d_model // 16),
+        "gemm_qkvab": ("tensor", 2.0 * M * N1 * d_model),
+        "delta_rule": ("hbm", M * (2 * HK + HV) * 2 + 2 * M * H * 4 + M * HV * 2 + B * H * dk * dv * 4),
+        "quant_o": ("hbm", M * HV * 2 + M * HV // 2 + M * HV // 16),
+        "gemm_out": ("tensor", 2.0 * M * d_model * HV),
+    }
+
+
+def traffic_from_profiles(kernel):
+    """dram bytes per launch from the committed ncu summary, if the kernel
+    source it was taken from is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "nvfp4_w4a4_gated_quant_b200", "csrc", rec["source"])
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if h == rec["source_sha"] else None
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from nvfp4_w4a4_gated_quant_b200 import _lib, inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    W = WORKLOAD
+    B, T, D, H, dk, dv = W["B"], W["T"], W["d_model"], W["H"], W["dk"], W["dv"]
+    M, HK, HV = B * T, H * dk, H * dv
+    d = inputs.layer_inputs(B, T, D, H, dk, dv, seed=3 + rank)
+    stream = torch.cuda.current_stream()
+    lw = _lib.QuantizedLayerWeights(d["W"], d["A_log"], d["dt_bias"], H, dk, dv, device=dev)
+    x_host = torch.from_numpy(d["x"]).to(torch.bfloat16).pin_memory()
+    x = x_host.to(dev)
+    y = torch.empty_like(x)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    y_host = torch.empty(x.shape, dtype=torch.bfloat16).pin_memory()
+    cfg = _lib.layer_cfg(B, T, D, H, dk, dv)
+    ws = torch.empty(_lib.gdn_layer_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    off = _lib.gdn_layer_workspace_offsets(cfg)
+
+    def layer_step():
+        _lib.gdn_layer_fwd(lw, x, y=y, S_T=S_T, ws=ws)
+
+    # views of the workspace for the staged run (same calls the layer makes)
+    u8 = ws
+    NQKV = 2 * HK + HV
+    x_codes = u8[off[_lib.WS_X_CODES]:].narrow(0, 0, M * D // 2).view(M, D // 2)
+    x_scales = u8[off[_lib.WS_X_SCALES]:].narrow(0, 0, _lib.scales_tiled_bytes(M, D))
+    x_g = u8[off[_lib.WS_X_G]:].narrow(0, 0, 4).view(torch.float32)
+    qkv = u8[off[_lib.WS_QKV]:].narrow(0, 0, M * NQKV * 2).view(torch.bfloat16).view(M, NQKV)
+    la = u8[off[_lib.WS_LOG_ALPHA]:].narrow(0, 0, M * H * 4).view(torch.float32).view(M, H)
+    be = u8[off[_lib.WS_BETA]:].narrow(0, 0, M * H * 4).view(torch.float32).view(M, H)
+    o = u8[off[_lib.WS_O]:].narrow(0, 0, M * HV * 2).view(torch.bfloat16).view(B, T, H, dv)
+    o_codes = u8[off[_lib.WS_O_CODES]:].narrow(0, 0, M * HV // 2).view(M, HV // 2)
+    o_scales = u8[off[_lib.WS_O_SCALES]:].narrow(0, 0, _lib.scales_tiled_bytes(M, HV))
+    o_g = u8[off[_lib.WS_O_G]:].narrow(0, 0, 4).view(torch.float32)
+    qws = u8[off[_lib.WS_QUANT]:].narrow(0, 0, 256)
+    segs = [
+        {"n_begin": 0, "n_end": HK, "kind": _lib.EPI_STORE_BF16, "g_b": lw.g["q"], "out": qkv, "ld_out": NQKV},
+        {"n_begin": HK, "n_end": 2 * HK, "kind": _lib.EPI_STORE_BF16, "g_b": lw.g["k"], "out": qkv, "out_offset": HK,
+         "ld_out": NQKV},
+        {"n_begin": 2 * HK, "n_end": NQKV, "kind": _lib.EPI_STORE_BF16, "g_b": lw.g["v"], "out": qkv,
+         "out_offset": 2 * HK, "ld_out": NQKV},
+        {"n_begin": NQKV, "n_end": NQKV + H, "kind": _lib.EPI_LOG_ALPHA, "g_b": lw.g["a"], "out": la, "ld_out": H,
+         "A_log": lw.A_log, "dt_bias": lw.dt_bias},
+        {"n_begin": NQKV + H, "n_end": NQKV + 2 * H, "kind": _lib.EPI_BETA, "g_b": lw.g["b"], "out": be, "ld_out": H},
+    ]
+    qv = qkv.view(B, T, NQKV)
+    stages = [
+        ("quant_x", lambda: _lib.gdn_quantize_nvfp4(x.view(M, D), codes=x_codes, scales=x_scales, g_out=x_g, ws=qws)),
+        ("gemm_qkvab", lambda: _lib.gdn_gemm_nvfp4(x_codes, x_scales, x_g, lw.codes, lw.scales, M, NQKV + 2 * H, D,
+                                                  segs)),
+        ("delta_rule", lambda: _lib.gdn_delta_rule_fwd(
+            qv[:, :, :HK].view(B, T, H, dk), qv[:, :, HK:2 * HK].view(B, T, H, dk),
+            qv[:, :, 2 * HK:].view(B, T, H, dv), la.view(B, T, H), be.view(B, T, H), o=o, S_T=S_T)),
+        ("quant_o", lambda: _lib.gdn_quantize_nvfp4(o.view(M, HV), codes=o_codes, scales=o_scales, g_out=o_g, ws=qws)),
+        ("gemm_out", lambda: _lib.gemm_bf16(o_codes, o_scales, o_g, lw.out_codes, lw.out_scales, lw.g["out"], M, D, HV,
+                                            out=y.view(M, D))),
+    ]
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        layer_step()
+        for _, fn in stages:
+            fn()
+    _lib.stream_check()
+
+    # ---- timed: the product call on device-resident inputs
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            layer_step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    _lib.stream_check()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+
+    # ---- stage breakdown: the same calls one by one, events between them
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        sev[i][0].record(stream)
+        for j, (_, fn) in enumerate(stages):
+            fn()
+            sev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    _lib.stream_check()
+    stage_ms = {name: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(args.steps))
+                for j, (name, _) in enumerate(stages)}
+
+    # ---- end to end through the public call with host buffers
+    eev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier()
+    torch.cuda.synchronize()
+    eev[0].record(stream)
+    for _ in range(args.steps):
+        x.copy_(x_host, non_blocking=True)
+        layer_step()
+        y_host.copy_(y, non_blocking=True)
+    eev[1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(eev[0].elapsed_time(eev[1])) / args.steps
+
+    # ---- standalone kernels of the GEMM and scan workloads (context keys)
+    kernels = standalone_kernels(args, torch, _lib, inputs, dev, stream) if rank == 0 and not args.skip_kernels else {}
+
+    clk = clocks.summary()
+    tokens_per_step = M * world
+    value = tokens_per_step / (ms_per_step / 1e3)
+    pk = peaks()
+    fp4_peak = 4.0 * pk["bf16_tflops_sustained"]           # FP4 dense = 4x bf16 (nominal ratio)
+    costs = stage_costs(B, T, D, H, dk, dv)
+    stage_out = {}
+    for name, ms in stage_ms.items():
+        bound, work = costs[name]
+        if bound == "hbm":
+            ach = work / (ms / 1e3) / 1e9
+            stage_out[name] = {"us": round(ms * 1e3, 1), "bound": "hbm", "achieved_GBps": round(ach, 1),
+                               "frac": round(ach / pk["hbm_gbs"], 4)}
+        else:
+            ach = work / (ms / 1e3) / 1e12
+            stage_out[name] = {"us": round(ms * 1e3, 1), "bound": "tensor", "achieved_TFLOPs": round(ach, 1),
+                               "frac": round(ach / fp4_peak, 4)}
+    dom = max(stage_ms, key=stage_ms.get)
+    bound, work = costs[dom]
+    kname = {"quant_x": "quant_kernel", "quant_o": "quant_kernel", "gemm_qkvab": "gemm_nvfp4_kernel",
+             "gemm_out": "gemm_nvfp4_kernel", "delta_rule": "delta_rule_kernel"}[dom]
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": round(work / (stage_ms[dom] / 1e3) / 1e9, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(work / (stage_ms[dom] / 1e3) / 1e12, 1), "peak": fp4_peak,
+                "unit": "TFLOP/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["traffic"] = traffic_from_profiles(kname)
+    roof["kernel"] = f"{dom} ({kname})"
+    roof["peak_source"] = (f"{pk['source']}: " + ("hbm_gbs" if bound == "hbm" else
+                                                  "4 x bf16_tflops_sustained (FP4 = 4x bf16 nominal)"))
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3, fp32 acc); scan fp16 mma, fp32 state",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, **W, "tokens_per_step_per_gpu": M,
+                   "l2": "inputs exceed L2 (x 335 MB, q/k/v 805 MB per step); no flush",
+                   "parallelism": f"replicas x{world} (independent batches per GPU)"},
+        "e2e": {"value": round(tokens_per_step / (e2e_ms / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
+        "gpu_launches": 7 * args.steps,
+        "roofline": roof,
+        "stages": stage_out,
+        "clocks": clk,
+        "step_ms_min_max": [round(min(step_ms), 4), round(max(step_ms), 4)],
+    }
+    if kernels:
+        line["kernels"] = kernels
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline(seconds_budget=args.cpu_seconds)
+    return line
+
+
+def standalone_kernels(args, torch, _lib, inputs, dev, stream, which=None):
+    """The GEMM workload (8192 x 12288 x 5120, bf16 out) and the scan workload
+    (T=32768, H=16, d=128) timed alone, for their own roofline fractions."""
+    out = {}
+    pk = peaks()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(args.steps, 10) if which is None else args.steps
+    if which == "scan":
+        return standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps)
+    rng = np.random.default_rng(1)
+    M, N, K = 8192, 12288, 5120
+    x = torch.from_numpy(inputs.activations(rng, (M, K))).to(dev).to(torch.bfloat16)
+    w = torch.randn((N, K), generator=torch.Generator().manual_seed(1)).mul_(0.02).to(dev)
+    xc, xs, gx = _lib.gdn_quantize_nvfp4(x)
+    wc, wsc, gw = _lib.gdn_quantize_nvfp4(w)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        _lib.gemm_bf16(xc, xs, gx, wc, wsc, gw, M, N, K, out=y)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        _lib.gemm_bf16(xc, xs, gx, wc, wsc, gw, M, N, K, out=y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    tf = 2.0 * M * N * K / (ms / 1e3) / 1e12
+    out["gemm_8192x12288x5120"] = {"us": round(ms * 1e3, 1), "TFLOPs": round(tf, 1),
+                                   "frac_fp4_burst": round(tf / (4 * pk["bf16_tflops"]), 4),
+                                   "frac_fp4_nominal_9PF": round(tf / 9000.0, 4)}
+    del x, w, xc, xs, wc, wsc, y
+    if which == "gemm":
+        return out
+    return standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps)
+
+
+def standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps):
+    B, T, H, d = 1, 32768, 16, 128
+    g = torch.Generator().manual_seed(2)
+    q = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    la = (-torch.rand((B, T, H), generator=g) * 1.5).to(dev)
+    be = torch.rand((B, T, H), generator=g).to(dev)
+    o = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = 4 * B * T * H * d * 2 + 2 * B * T * H * 4 + B * H * d * d * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["scan_T32768_H16_d128"] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1),
+                                   "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    return out
+
+
+# ------------------------------------------------------------ CPU baseline --
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_sample(T_sample):
+    """The oracle layer on the first T_sample tokens of one sequence of the
+    layer workload (weights quantized by the oracle once, outside the timing)."""
+    from oracle.layer import layer_forward, quantize_weights
+    from nvfp4_w4a4_gated_quant_b200 import inputs
+    W = WORKLOAD
+    rng = np.random.default_rng(3)
+    x = inputs.activations(rng, (1, T_sample, W["d_model"]))
+    Wd = {n: inputs.weight(rng, r, c) for n, (r, c) in {
+        "q": (W["H"] * W["dk"], W["d_model"]), "k": (W["H"] * W["dk"], W["d_model"]),
+        "v": (W["H"] * W["dv"], W["d_model"]), "a": (W["H"], W["d_model"]), "b": (W["H"], W["d_model"]),
+        "out": (W["d_model"], W["H"] * W["dv"])}.items()}
+    A = rng.uniform(-2, 1, W["H"])
+    dt = rng.uniform(-1, 1, W["H"])
+    Wq = quantize_weights(Wd)
+    return lambda: layer_forward(x, Wq, A, dt, W["H"], W["dk"], W["dv"])
+
+
+def cpu_baseline(seconds_budget=20.0, T_sample=CPU_SAMPLE_T):
+    fn = _oracle_sample(T_sample)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        if time.perf_counter() - t0 > seconds_budget / 2 or n >= 3:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(T_sample / dt, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{T_sample} tokens of 1 sequence of the layer workload (d_model 5120, H 32, d 128), "
+                      f"{n} run(s), mean {dt:.2f} s each; weights quantized outside the timing"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    fn = _oracle_sample(CPU_SAMPLE_T)
+    for _ in range(min(args.warmup, 1)):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = CPU_SAMPLE_T / dt
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (quantizer f32)", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, **WORKLOAD},
+        "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                         "sample": f"each step: the oracle layer on {CPU_SAMPLE_T} tokens of 1 sequence"},
+        "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the oracle CPU baseline")
+    ap.add_argument("--skip-kernels", action="store_true", help="omit the standalone GEMM / scan timings")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--only", choices=["gemm", "scan"], default=None,
+                    help="time only the standalone GEMM or scan workload (profiling target)")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if args.only:
+        import torch
+        from nvfp4_w4a4_gated_quant_b200 import _lib, inputs
+        torch.cuda.set_device(local_rank)
+        k = standalone_kernels(args, torch, _lib, inputs, torch.device("cuda", local_rank),
+                               torch.cuda.current_stream(), which=args.only)
+        print(json.dumps({"only": args.only, "kernels": k}), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    line = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
