@@ -13,13 +13,22 @@
 //                 (128-byte rows, 128B swizzle) plus their E4M3 scale blocks
 //                 (untiled bulk copies of the tensor-core scale layout) into a
 //                 4-stage shared-memory ring.  No multicast.
-//   warp 1        TMEM owner and MMA issuer: copies each stage's scales to
-//                 TMEM (tcgen05.cp 32x128b.warpx4), then issues
+//   warps 12..15  scale loaders, one per 32-lane TMEM quarter: each stage's
+//                 scales go from shared memory to a double-buffered TMEM
+//                 region with tcgen05.st (replicated into the four quarters,
+//                 the layout the block-scaled MMA reads).  Doing this with
+//                 warp stores keeps the copies off the MMA pipe, where
+//                 tcgen05.cp serialises with the MMAs.
+//   warp 1        TMEM owner and MMA issuer:
 //                 tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128,
 //                 N=256, K=64) into a 128 x 256 FP32 accumulator in TMEM;
 //                 tcgen05.commit frees the stage / publishes the tile.
-//   warps 4..11   epilogue: tcgen05.ld of 32-column slices, the per-segment
-//                 scale, then bf16 / FP32 stores or the gate functions.
+//   warps 4..11   epilogue: tcgen05.ld of 32-column slices.  On tiles whose
+//                 128 columns per warp fall in one bf16 segment the values
+//                 are scaled and packed to bf16 in registers, the accumulator
+//                 is released, and the stores overlap the next tile's MMAs;
+//                 other tiles (segment edges, gates, FP32 outputs) take the
+//                 per-column path.
 // Every mbarrier wait is bounded; a wait that runs out records
 // GDN_ERR_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
 #include <cuda.h>
@@ -43,16 +52,17 @@ constexpr int A_BYTES = BM * BK / 2;    // 16 KiB
 constexpr int B_BYTES = BN * BK / 2;    // 32 KiB
 constexpr int SFA_BYTES = (BK / KSTEP) * 512;          // 2 KiB
 constexpr int SFB_BYTES = (BN / 128) * (BK / KSTEP) * 512;  // 4 KiB
-constexpr int NUM_THREADS = 384;
+constexpr int NUM_THREADS = 512;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
+constexpr int SF_WARP0 = 12;            // warps 12..15: scale loaders
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;         // 256 FP32 columns
-constexpr uint32_t SFA_COL = 256;       // 4 k-steps x 4 columns
-constexpr uint32_t SFB_COL = 272;       // 4 k-steps x 8 columns
+constexpr uint32_t SF_COL = 256;        // two buffers of 48 columns:
+constexpr uint32_t SF_BUF = 48;         //   +0: A, 4 k-steps x 4; +16: B, 4 k-steps x 8
 
 constexpr size_t SMEM_BYTES =
-    1024 /*alignment slack*/ + (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 256;
+    1024 /*alignment slack*/ + (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 512;
 
 struct Segment {
   int n_begin, n_end, kind;
@@ -82,13 +92,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset
   d |= (uint64_t)1 << 46;                 // descriptor version (sm_100)
   d |= (uint64_t)2 << 61;                 // 128-byte swizzle
-  return d;
-}
-// Scale block for tcgen05.cp: 32 rows of 16 bytes, 8-row groups 128 B apart.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)(128 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
   return d;
 }
 // Instruction descriptor: E2M1 x E2M1, UE4M3 scales, FP32 accumulate,
@@ -144,7 +147,9 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
+  uint64_t* sf_full = empty + STAGES;   // [2] scales of a stage are in TMEM buffer
+  uint64_t* sf_free = sf_full + 2;      // [2] the MMAs that read a buffer are done
+  uint64_t* acc_full = sf_free + 2;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
@@ -156,6 +161,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sf_full[b], 4);
+      mbar_init(&sf_free[b], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, NUM_EPI_WARPS);
@@ -214,35 +223,77 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         }
     }
     __syncwarp();
+  } else if (warp >= SF_WARP0) {
+    // ------------------------------------------------------- scale loaders
+    // Warp w writes TMEM lanes 32*(w%4) .. +31.  Column c of k-step j holds,
+    // in lane l, the four scales of row (l%32) + 32c: the 16 bytes at
+    // (l%32)*16 of the k-step's 512-byte block, identical in every quarter.
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t buf = it & 1;
+        bool got = true;
+        if (lane == 0)
+          got = wait_or_abort(&sf_free[buf], ((it >> 1) & 1) ^ 1, p.status, abort_flag) &&
+                wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag);
+        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) { ok = false; break; }
+        tc_fence_after();
+        uint32_t ra[16], rb[16], rc[16];
+        const uint4* fa = reinterpret_cast<const uint4*>(sSFA + s * SFA_BYTES) + lane;
+        const uint4* fb = reinterpret_cast<const uint4*>(sSFB + s * SFB_BYTES) + lane;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 a4 = fa[j * 32];             // k-step j, A
+          ra[4 * j + 0] = a4.x; ra[4 * j + 1] = a4.y; ra[4 * j + 2] = a4.z; ra[4 * j + 3] = a4.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint4 b4 = fb[(h * 4 + j) * 32];  // k-step j, B rows 128h .. 128h+127
+            uint32_t* dst = (j < 2 ? rb : rc) + (j & 1) * 8 + h * 4;
+            dst[0] = b4.x; dst[1] = b4.y; dst[2] = b4.z; dst[3] = b4.w;
+          }
+        }
+        const uint32_t col = tmem + lane_base + SF_COL + buf * SF_BUF;
+        tmem_st_32x32b_x16(col, ra);
+        tmem_st_32x32b_x16(col + 16, rb);
+        tmem_st_32x32b_x16(col + 32, rc);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[buf]);
+      }
+    }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
       uint32_t it = 0, tile_iter = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
-        const int nb = tile / p.num_m;
-        const int nh = min(2, sf_blocks_n - 2 * nb);
         if (!wait_or_abort(acc_empty, (tile_iter & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
-          const uint32_t round = it / STAGES;
-          if (!wait_or_abort(&full[s], round & 1, p.status, abort_flag)) { ok = false; break; }
+          const uint32_t buf = it & 1;
+          if (!wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag) ||
+              !wait_or_abort(&sf_full[buf], (it >> 1) & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
-          const uint32_t sfa_s = smem_u32(sSFA + s * SFA_BYTES);
-          const uint32_t sfb_s = smem_u32(sSFB + s * SFB_BYTES);
-          for (int j = 0; j < nks; ++j) {
-            tc_cp_32x128b_warpx4(tmem + SFA_COL + j * 4, desc_sf(sfa_s + j * 512));
-            for (int h = 0; h < nh; ++h)
-              tc_cp_32x128b_warpx4(tmem + SFB_COL + j * 8 + h * 4, desc_sf(sfb_s + (h * 4 + j) * 512));
-          }
           const uint32_t a_s = smem_u32(sA + s * A_BYTES);
           const uint32_t b_s = smem_u32(sB + s * B_BYTES);
+          const uint32_t sfa = tmem + SF_COL + buf * SF_BUF;
           for (int j = 0; j < nks; ++j)
-            tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc,
-                        tmem + SFA_COL + j * 4, tmem + SFB_COL + j * 8, (kb > 0 || j > 0) ? 1u : 0u);
+            tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc, sfa + j * 4,
+                        sfa + 16 + j * 8, (kb > 0 || j > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
+          tc_commit(&sf_free[buf]);
         }
         if (ok) tc_commit(acc_full);
       }
@@ -263,38 +314,56 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       tc_fence_after();
       const int m = mb * BM + quad * 32 + lane;
       const float g_a = *p.g_a;
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        const int col0 = half * 128 + c * 32;
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + col0, r);
-        tc_wait_ld();
-        if (c == 3) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
-        }
-        const int n0 = nb * BN + col0;
-        if (m >= p.M || n0 >= p.N) continue;
-        const int s0 = find_segment(p, n0);
+      const int nw0 = nb * BN + half * 128;   // first column of this warp
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
+      // Fast path: all 128 columns inside one bf16 segment with 16-byte
+      // aligned rows -> pack, release the accumulator, then store.
+      bool fast = false;
+      int s0 = 0;
+      if (nw0 < p.N) {
+        s0 = find_segment(p, nw0);
         const Segment& sg = p.segs[s0];
-        const bool whole = (n0 + 31 < sg.n_end) && (n0 + 31 < p.N);
-        const int64_t off = (int64_t)m * sg.ld_out + (n0 - sg.n_begin);
-        if (whole && sg.kind == GDN_EPI_STORE_BF16 && ((reinterpret_cast<uintptr_t>(sg.out) + off * 2) % 16) == 0) {
-          const float alpha = __fmul_rn(g_a, *sg.g_b);
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(sg.out) + off);
+        fast = sg.kind == GDN_EPI_STORE_BF16 && nw0 + 127 < sg.n_end && nw0 + 127 < p.N &&
+               (sg.ld_out % 8) == 0 && ((reinterpret_cast<uintptr_t>(sg.out) + (int64_t)(nw0 - sg.n_begin) * 2) % 16) == 0;
+      }
+      if (fast) {
+        const Segment& sg = p.segs[s0];
+        const float alpha = __fmul_rn(g_a, *sg.g_b);
+        uint32_t pk[64];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c * 32, r);
+          tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float y0 = __fmul_rn(__uint_as_float(r[v * 8 + 2 * e]), alpha);
-              const float y1 = __fmul_rn(__uint_as_float(r[v * 8 + 2 * e + 1]), alpha);
-              w[e] = f32_to_bf16_bits(y0) | (f32_to_bf16_bits(y1) << 16);
-            }
-            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 16; ++e) {
+            const float y0 = __fmul_rn(__uint_as_float(r[2 * e]), alpha);
+            const float y1 = __fmul_rn(__uint_as_float(r[2 * e + 1]), alpha);
+            pk[c * 16 + e] = f32_to_bf16_bits(y0) | (f32_to_bf16_bits(y1) << 16);
           }
-        } else {
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        if (m < p.M) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(sg.out) + (int64_t)m * sg.ld_out +
+                                                (nw0 - sg.n_begin));
+#pragma unroll
+          for (int v = 0; v < 16; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      } else {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(tbase + c * 32, r);
+          tc_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          const int n0 = nw0 + c * 32;
+          if (m >= p.M || n0 >= p.N) continue;
 #pragma unroll 1
           for (int i = 0; i < 32; ++i) {
             const int n = n0 + i;
