@@ -10,25 +10,32 @@
 //
 // Design (one CTA per SM, persistent over 128 x 256 output tiles, M fastest):
 //   warp 0        TMA producer: A tile 128 x 256 fp4 and B tile 256 x 256 fp4
-//                 (128-byte rows, 128B swizzle) plus their E4M3 scale blocks
-//                 (untiled bulk copies of the tensor-core scale layout) into a
-//                 4-stage shared-memory ring.  No multicast.
-//   warps 12..15  scale loaders, one per 32-lane TMEM quarter: each stage's
-//                 scales go from shared memory to a double-buffered TMEM
-//                 region with tcgen05.st (replicated into the four quarters,
-//                 the layout the block-scaled MMA reads).  Doing this with
-//                 warp stores keeps the copies off the MMA pipe, where
+//                 (128-byte rows, 128B swizzle) plus the E4M3 scale blocks
+//                 they need (untiled bulk copies of the tensor-core scale
+//                 layout) into a 4-stage shared-memory ring.  No multicast.
+//   warps 12..15  scale loaders, one per 32-lane TMEM quarter: as soon as a
+//                 stage lands they read its scales from shared memory into
+//                 registers, then, once one of three TMEM scale buffers is
+//                 free, write them with tcgen05.st, replicated into the four
+//                 quarters (the layout the block-scaled MMA reads).  Warp
+//                 stores keep these copies off the MMA pipe, where
 //                 tcgen05.cp serialises with the MMAs.
 //   warp 1        TMEM owner and MMA issuer:
 //                 tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128,
 //                 N=256, K=64) into a 128 x 256 FP32 accumulator in TMEM;
-//                 tcgen05.commit frees the stage / publishes the tile.
-//   warps 4..11   epilogue: tcgen05.ld of 32-column slices.  On tiles whose
-//                 128 columns per warp fall in one bf16 segment the values
-//                 are scaled and packed to bf16 in registers, the accumulator
-//                 is released, and the stores overlap the next tile's MMAs;
-//                 other tiles (segment edges, gates, FP32 outputs) take the
-//                 per-column path.
+//                 tcgen05.commit frees smem stages, scale buffers and tiles.
+//                 (The MMA's shared-memory operand reads plus the TMA writes
+//                 come close to the SM's shared-memory bandwidth; the widest
+//                 N tile re-reads A the least.)
+//   warps 4..11   epilogue: tcgen05.ld of 32-column slices with the
+//                 per-segment scale (g_a * g_b, precomputed into a
+//                 shared-memory segment table at kernel start).  When a
+//                 warp's 128 columns lie in one bf16 segment they are packed
+//                 to bf16 in registers, the accumulator is released at once
+//                 and the stores overlap the next tile's MMAs; other tiles
+//                 (segment edges, gates, FP32 outputs) take the per-column
+//                 path and release after their last load.
+// TMEM: accumulator at columns 0..255, scale buffers at 256 + 48b.
 // Every mbarrier wait is bounded; a wait that runs out records
 // GDN_ERR_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
 #include <cuda.h>
@@ -50,19 +57,34 @@ constexpr int KSTEP = 64;               // K of one MMA
 constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK / 2;    // 16 KiB
 constexpr int B_BYTES = BN * BK / 2;    // 32 KiB
-constexpr int SFA_BYTES = (BK / KSTEP) * 512;          // 2 KiB
-constexpr int SFB_BYTES = (BN / 128) * (BK / KSTEP) * 512;  // 4 KiB
 constexpr int NUM_THREADS = 512;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int SF_WARP0 = 12;            // warps 12..15: scale loaders
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;         // 256 FP32 columns
-constexpr uint32_t SF_COL = 256;        // two buffers of 48 columns:
+constexpr uint32_t ACC_COL = 0;         // one accumulator of BN FP32 columns
+constexpr int SF_NBUF = 5;
+constexpr uint32_t SF_COL = BN;         // five buffers of 48 columns:
 constexpr uint32_t SF_BUF = 48;         //   +0: A, 4 k-steps x 4; +16: B, 4 k-steps x 8
+constexpr uint32_t SFB_OFF = 16;
+constexpr uint32_t SFB_PER_K = BN / 32;
+static_assert(SF_COL + SF_NBUF * SF_BUF <= TMEM_COLS, "TMEM budget");
 
-constexpr size_t SMEM_BYTES =
-    1024 /*alignment slack*/ + (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 512;
+struct SegSmem {
+  int n_begin, n_end, kind, pad;
+  float alpha;            // g_a * g_b of the segment
+  int64_t ld_out;
+  void* out;
+  const float* A_log;
+  const float* dt_bias;
+};
+
+constexpr int SFA_BYTES = (BK / KSTEP) * 512;      // 2 KiB
+constexpr int SFB_BYTES = 2 * (BK / KSTEP) * 512;  // two 128-row scale blocks, 4 KiB
+
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ +
+                              (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 512 +
+                              GDN_MAX_SEGMENTS * sizeof(SegSmem);
 
 struct Segment {
   int n_begin, n_end, kind;
@@ -95,7 +117,7 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   return d;
 }
 // Instruction descriptor: E2M1 x E2M1, UE4M3 scales, FP32 accumulate,
-// both operands K-major, M = 128, N = 256, dense, K = 64.
+// both operands K-major, M = 128, N = BN, dense, K = 64.
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
@@ -109,14 +131,14 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
   return false;
 }
 
-__device__ __forceinline__ int find_segment(const Params& p, int n) {
+__device__ __forceinline__ int find_segment(const SegSmem* segs, int n_segs, int n) {
   int s = 0;
 #pragma unroll 1
-  while (s + 1 < p.n_segs && n >= p.segs[s].n_end) ++s;
+  while (s + 1 < n_segs && n >= segs[s].n_end) ++s;
   return s;
 }
 
-__device__ __forceinline__ void epilogue_store_one(const Segment& sg, int m, int n, float y) {
+__device__ __forceinline__ void epilogue_store_one(const SegSmem& sg, int m, int n, float y) {
   const int64_t off = (int64_t)m * sg.ld_out + (n - sg.n_begin);
   switch (sg.kind) {
     case GDN_EPI_STORE_BF16:
@@ -136,6 +158,10 @@ __device__ __forceinline__ void epilogue_store_one(const Segment& sg, int m, int
   }
 }
 
+__device__ __forceinline__ uint32_t word(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                   const __grid_constant__ Params p) {
@@ -145,11 +171,12 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSFA = sB + STAGES * B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  SegSmem* segs = reinterpret_cast<SegSmem*>(sSFB + STAGES * SFB_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(segs + GDN_MAX_SEGMENTS);
   uint64_t* empty = full + STAGES;
-  uint64_t* sf_full = empty + STAGES;   // [2] scales of a stage are in TMEM buffer
-  uint64_t* sf_free = sf_full + 2;      // [2] the MMAs that read a buffer are done
-  uint64_t* acc_full = sf_free + 2;
+  uint64_t* sf_full = empty + STAGES;      // [3] a scale buffer is filled
+  uint64_t* sf_free = sf_full + SF_NBUF;   // [3] the MMAs that read a buffer are done
+  uint64_t* acc_full = sf_free + SF_NBUF;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_ptr + 1);
@@ -162,7 +189,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < SF_NBUF; ++b) {
       mbar_init(&sf_full[b], 4);
       mbar_init(&sf_free[b], 1);
     }
@@ -170,6 +197,18 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     mbar_init(acc_empty, NUM_EPI_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (threadIdx.x < p.n_segs) {
+    const Segment& g = p.segs[threadIdx.x];
+    SegSmem& d = segs[threadIdx.x];
+    d.n_begin = g.n_begin;
+    d.n_end = g.n_end;
+    d.kind = g.kind;
+    d.alpha = __fmul_rn(*p.g_a, *g.g_b);
+    d.ld_out = g.ld_out;
+    d.out = g.out;
+    d.A_log = g.A_log;
+    d.dt_bias = g.dt_bias;
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmap_a);
@@ -183,6 +222,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr;
+  const int n_segs = p.n_segs;
 
   const int num_kb = (p.K + BK - 1) / BK;
   const int ksteps_total = p.K / KSTEP;
@@ -198,7 +238,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         const int mb = tile % p.num_m, nb = tile / p.num_m;
-        const int nh = min(2, sf_blocks_n - 2 * nb);
+        const int b0 = (nb * BN) / 128;                 // first 128-row scale block of B
+        const int nh = min(2, sf_blocks_n - b0);
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t round = it / STAGES;
@@ -210,7 +251,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           tma_load_2d(sB + s * B_BYTES, &tmap_b, &full[s], kb * (BK / 2), nb * BN);
           bulk_load(sSFA + s * SFA_BYTES, p.sfa + ((int64_t)mb * p.kc + kb * 4) * 512, nks * 512, &full[s]);
           for (int h = 0; h < nh; ++h)
-            bulk_load(sSFB + s * SFB_BYTES + h * 2048, p.sfb + ((int64_t)(2 * nb + h) * p.kc + kb * 4) * 512,
+            bulk_load(sSFB + s * SFB_BYTES + h * 2048, p.sfb + ((int64_t)(b0 + h) * p.kc + kb * 4) * 512,
                       nks * 512, &full[s]);
           issued[s] = true;
           last_round[s] = round;
@@ -225,43 +266,48 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     __syncwarp();
   } else if (warp >= SF_WARP0) {
     // ------------------------------------------------------- scale loaders
-    // Warp w writes TMEM lanes 32*(w%4) .. +31.  Column c of k-step j holds,
-    // in lane l, the four scales of row (l%32) + 32c: the 16 bytes at
-    // (l%32)*16 of the k-step's 512-byte block, identical in every quarter.
+    // Warp w writes TMEM lanes 32*(w%4) .. +31.  For k-step j, column c of
+    // the A part holds in lane l the four scales of row (l%32) + 32c: the
+    // 16 bytes at (l%32)*16 of the k-step's 512-byte block.  The B part has
+    // BN/32 columns; its rows 32c + l of the tile form 32-row group
+    // g = nb*BN/32 + c, which sits in scale block g/4 (relative to the first
+    // block the tile touches) as word g%4 of the lane's 16 bytes.
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
         const int s = it % STAGES;
-        const uint32_t buf = it & 1;
+        const uint32_t buf = it % SF_NBUF;
         bool got = true;
-        if (lane == 0)
-          got = wait_or_abort(&sf_free[buf], ((it >> 1) & 1) ^ 1, p.status, abort_flag) &&
-                wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag);
+        if (lane == 0) got = wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag);
         if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) { ok = false; break; }
-        tc_fence_after();
-        uint32_t ra[16], rb[16], rc[16];
         const uint4* fa = reinterpret_cast<const uint4*>(sSFA + s * SFA_BYTES) + lane;
         const uint4* fb = reinterpret_cast<const uint4*>(sSFB + s * SFB_BYTES) + lane;
+        uint32_t ra[16], rb[16], rc[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint4 a4 = fa[j * 32];             // k-step j, A
+          const uint4 a4 = fa[j * 32];
           ra[4 * j + 0] = a4.x; ra[4 * j + 1] = a4.y; ra[4 * j + 2] = a4.z; ra[4 * j + 3] = a4.w;
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+          const uint4 x0 = fb[j * 32];          // block 0, k-step j
+          const uint4 x1 = fb[128 + j * 32];    // block 1, k-step j
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 b4 = fb[(h * 4 + j) * 32];  // k-step j, B rows 128h .. 128h+127
-            uint32_t* dst = (j < 2 ? rb : rc) + (j & 1) * 8 + h * 4;
-            dst[0] = b4.x; dst[1] = b4.y; dst[2] = b4.z; dst[3] = b4.w;
+          for (int c = 0; c < (int)SFB_PER_K; ++c) {
+            const uint32_t v = word(c < 4 ? x0 : x1, c & 3);   // tile starts on a scale block
+            const int idx = j * SFB_PER_K + c;
+            if (idx < 16) rb[idx] = v; else rc[idx - 16] = v;
           }
         }
+        if (lane == 0) got = wait_or_abort(&sf_free[buf], ((it / SF_NBUF) & 1) ^ 1, p.status, abort_flag);
+        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) { ok = false; break; }
+        tc_fence_after();
         const uint32_t col = tmem + lane_base + SF_COL + buf * SF_BUF;
         tmem_st_32x32b_x16(col, ra);
-        tmem_st_32x32b_x16(col + 16, rb);
-        tmem_st_32x32b_x16(col + 32, rc);
+        tmem_st_32x32b_x16(col + SFB_OFF, rb);
+        tmem_st_32x32b_x16(col + SFB_OFF + 16, rc);
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -276,11 +322,12 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
         if (!wait_or_abort(acc_empty, (tile_iter & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t acc = tmem + ACC_COL;
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
-          const uint32_t buf = it & 1;
+          const uint32_t buf = it % SF_NBUF;
           if (!wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag) ||
-              !wait_or_abort(&sf_full[buf], (it >> 1) & 1, p.status, abort_flag)) {
+              !wait_or_abort(&sf_full[buf], (it / SF_NBUF) & 1, p.status, abort_flag)) {
             ok = false;
             break;
           }
@@ -288,10 +335,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
           const uint32_t a_s = smem_u32(sA + s * A_BYTES);
           const uint32_t b_s = smem_u32(sB + s * B_BYTES);
-          const uint32_t sfa = tmem + SF_COL + buf * SF_BUF;
+          const uint32_t sf = tmem + SF_COL + buf * SF_BUF;
           for (int j = 0; j < nks; ++j)
-            tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc, sfa + j * 4,
-                        sfa + 16 + j * 8, (kb > 0 || j > 0) ? 1u : 0u);
+            tc_mma_nvf4(acc, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc, sf + j * 4,
+                        sf + SFB_OFF + j * SFB_PER_K, (kb > 0 || j > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
           tc_commit(&sf_free[buf]);
         }
@@ -307,28 +354,27 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     uint32_t tile_iter = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
       const int mb = tile % p.num_m, nb = tile / p.num_m;
+      const int m = mb * BM + quad * 32 + lane;
+      const int nw0 = nb * BN + half * 128;   // first column of this warp
+      // resolve the segment before waiting: fast path when all 128 columns
+      // sit in one bf16 segment with 16-byte aligned rows
+      int s0 = 0;
+      bool fast = false;
+      if (nw0 < p.N) {
+        s0 = find_segment(segs, n_segs, nw0);
+        const SegSmem& sg = segs[s0];
+        fast = sg.kind == GDN_EPI_STORE_BF16 && nw0 + 127 < sg.n_end && nw0 + 127 < p.N && (sg.ld_out % 8) == 0 &&
+               ((reinterpret_cast<uintptr_t>(sg.out) + (int64_t)(nw0 - sg.n_begin) * 2) % 16) == 0;
+      }
       bool ok = true;
       if (lane == 0) ok = wait_or_abort(acc_full, tile_iter & 1, p.status, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      const int m = mb * BM + quad * 32 + lane;
-      const float g_a = *p.g_a;
-      const int nw0 = nb * BN + half * 128;   // first column of this warp
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
-      // Fast path: all 128 columns inside one bf16 segment with 16-byte
-      // aligned rows -> pack, release the accumulator, then store.
-      bool fast = false;
-      int s0 = 0;
-      if (nw0 < p.N) {
-        s0 = find_segment(p, nw0);
-        const Segment& sg = p.segs[s0];
-        fast = sg.kind == GDN_EPI_STORE_BF16 && nw0 + 127 < sg.n_end && nw0 + 127 < p.N &&
-               (sg.ld_out % 8) == 0 && ((reinterpret_cast<uintptr_t>(sg.out) + (int64_t)(nw0 - sg.n_begin) * 2) % 16) == 0;
-      }
       if (fast) {
-        const Segment& sg = p.segs[s0];
-        const float alpha = __fmul_rn(g_a, *sg.g_b);
+        const SegSmem& sg = segs[s0];
+        const float alpha = sg.alpha;
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -352,6 +398,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           for (int v = 0; v < 16; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       } else {
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           __syncwarp();
@@ -368,9 +415,8 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           for (int i = 0; i < 32; ++i) {
             const int n = n0 + i;
             if (n >= p.N) break;
-            const Segment& sgi = p.segs[find_segment(p, n)];
-            const float y = __fmul_rn(__uint_as_float(r[i]), __fmul_rn(g_a, *sgi.g_b));
-            epilogue_store_one(sgi, m, n, y);
+            const SegSmem& sgi = segs[find_segment(segs, n_segs, n)];
+            epilogue_store_one(sgi, m, n, __fmul_rn(__uint_as_float(r[i]), sgi.alpha));
           }
         }
       }
