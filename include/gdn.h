@@ -280,6 +280,32 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg,
                   const void* x, void* y, const float* S0, float* S_T,
                   void* ws, size_t ws_bytes, gdn_stream_t stream);
 
+/* ------------------------------------------------------------------------ *
+ * Allocation-free layer forward (no counterpart in the paper).
+ *
+ * For callers that cannot allocate device memory: code running while a CUDA
+ * graph is being captured without an allocator, plugins that receive only
+ * their input and output pointers, real-time paths with a fixed memory budget.
+ * Same computation, arguments and results as gdn_layer_fwd, except that the
+ * workspace is a static device array of GDN_LAYER_STATIC_WS_BYTES inside the
+ * library (present on every GPU that loads it, until the process exits).
+ *   - Sizes: a cfg whose gdn_layer_workspace_size() exceeds the array is
+ *     rejected with GDN_ERR_WORKSPACE (gdn_last_error() says by how much);
+ *     with d_model 5120, H 32, d 128 that is about 860 tokens per call.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - Concurrency: every call shares the one array, so calls that overlap on
+ *     the GPU (different streams, or threads without ordering) race; order
+ *     them on one stream.  The array keeps the last call's intermediates.
+ *   - Allocates nothing: no cudaMalloc / cudaFree or allocating routine.
+ * ------------------------------------------------------------------------ */
+#define GDN_LAYER_STATIC_WS_BYTES (32u << 20)
+
+int gdn_layer_fwd_static_ws(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg,
+                            const void* x, void* y, const float* S0, float* S_T,
+                            gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

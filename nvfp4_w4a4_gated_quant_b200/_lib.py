@@ -83,6 +83,8 @@ def lib():
             "gdn_layer_workspace_offsets": (ctypes.c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(c_i64)]),
             "gdn_layer_fwd": (ctypes.c_int, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerCfg), c_vp, c_vp,
                                              c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
+            "gdn_layer_fwd_static_ws": (ctypes.c_int, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerCfg), c_vp,
+                                                       c_vp, c_vp, c_vp, c_vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -95,7 +97,8 @@ def lib():
 EXPORTED = ("gdn_status_string", "gdn_last_error", "gdn_version", "gdn_stream_check",
             "gdn_quantize_workspace_size", "gdn_scales_tiled_bytes", "gdn_quantize_nvfp4", "gdn_gemm_nvfp4",
             "gdn_gates", "gdn_delta_rule_workspace_size", "gdn_delta_rule_fwd", "gdn_layer_workspace_size",
-            "gdn_layer_workspace_offsets", "gdn_layer_fwd")
+            "gdn_layer_workspace_offsets", "gdn_layer_fwd", "gdn_layer_fwd_static_ws")
+LAYER_STATIC_WS_BYTES = 32 << 20
 
 
 def check(status):
@@ -363,3 +366,26 @@ def gdn_layer_fwd(weights, x, S0=None, want_state=True, y=None, S_T=None, ws=Non
     check(lib().gdn_layer_fwd(ctypes.byref(ws_struct), ctypes.byref(cfg), _ptr(x), _ptr(y), _ptr(S0), _ptr(S_T),
                               _ptr(ws), ws.numel(), _stream(stream)))
     return y, S_T, ws
+
+
+def gdn_layer_fwd_static_ws(weights, x, S0=None, want_state=True, y=None, S_T=None, stream=None):
+    """The layer forward with its scratch in the library's static device
+    array (no workspace argument, nothing allocated by the call itself).
+    Returns (y, S_T).  Calls that overlap on the GPU race on the shared
+    array."""
+    _need(x, torch.bfloat16, "x")
+    if not x.is_contiguous() or x.dim() != 3:
+        raise ValueError("x must be a contiguous [B, T, d_model] tensor")
+    B, T, D = x.shape
+    cfg = layer_cfg(B, T, D, weights.H, weights.dk, weights.dv)
+    if y is None:
+        y = torch.empty_like(x)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, weights.H, weights.dk, weights.dv), dtype=torch.float32, device=x.device)
+    ws_struct = weights.struct()
+    st = lib().gdn_layer_fwd_static_ws(ctypes.byref(ws_struct), ctypes.byref(cfg), _ptr(x), _ptr(y), _ptr(S0),
+                                       _ptr(S_T), _stream(stream))
+    if st == 6:
+        raise GdnError(f"gdn status 6: {lib().gdn_last_error().decode()}")
+    check(st)
+    return y, S_T

@@ -1,5 +1,6 @@
 // C-ABI entry points: argument checks, workspace arithmetic, status plumbing.
 // Every check runs on the host before anything is enqueued.
+#include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -30,6 +31,13 @@ int current_device() {
 int record_cuda_error(cudaError_t err) {
   snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(err), cudaGetErrorString(err));
   return GDN_ERR_CUDA;
+}
+
+void set_error_text(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
 }
 
 int* device_status_word() {

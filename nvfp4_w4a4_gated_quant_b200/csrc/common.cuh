@@ -12,6 +12,8 @@ namespace gdn {
 // ---------------------------------------------------------------- host side
 // Records the CUDA error text for gdn_last_error() and maps it to a status.
 int record_cuda_error(cudaError_t err);
+// Sets the text gdn_last_error() returns (printf-style) for a non-CUDA error.
+void set_error_text(const char* fmt, ...);
 // Device address of the status word on the current device (nullptr on error).
 int* device_status_word();
 // Launch-error check after a <<<>>> launch.

@@ -2,6 +2,8 @@
 // the gates in its epilogue -> chunked delta rule -> quantize -> output GEMM.
 // Five kernel launches (plus one 4-byte memset per quantization) on the
 // caller's stream; every intermediate lives in the caller's workspace.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -124,3 +126,61 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free layer forward.
+//
+// Some callers cannot allocate device memory at all: code that runs while a
+// CUDA graph is being captured with no allocator to hand, plugins that are
+// given only their input and output pointers, and real-time paths whose
+// memory budget is fixed up front.  They call gdn_layer_fwd_static_ws, which
+// takes the layer's scratch (the intermediates between its kernels) from the
+// file-scope device array below instead of a caller workspace.
+//
+// The array is GDN_LAYER_STATIC_WS_BYTES (32 MiB) and lives on every GPU that
+// loads this library until the process exits.  Host code cannot pass the
+// array's name to a kernel: in host code the name is only a host-side stand-in
+// for the symbol.  The first call on each device therefore looks up the
+// array's device address with cudaGetSymbolAddress (with that device
+// current) and caches it.
+static __device__ __align__(256) uint8_t g_layer_static_ws[GDN_LAYER_STATIC_WS_BYTES];
+
+namespace {
+constexpr int kMaxDev = 64;
+void* g_static_ws_ptr[kMaxDev];
+std::mutex g_static_ws_mu;
+
+int static_ws_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  if (dev < 0 || dev >= kMaxDev) return GDN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_static_ws_mu);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_layer_static_ws);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    g_static_ws_ptr[dev] = p;
+  }
+  *out = g_static_ws_ptr[dev];
+  return GDN_OK;
+}
+}  // namespace
+
+extern "C" int gdn_layer_fwd_static_ws(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, const void* x,
+                                       void* y, const float* S0, float* S_T, gdn_stream_t stream) {
+  if (!w || !cfg_ok(cfg)) return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_layer_workspace_size(cfg);
+  if (need > (size_t)GDN_LAYER_STATIC_WS_BYTES) {
+    set_error_text("layer workspace of %zu bytes exceeds the %zu-byte static scratch", need,
+                   (size_t)GDN_LAYER_STATIC_WS_BYTES);
+    return GDN_ERR_WORKSPACE;
+  }
+  void* ws = nullptr;
+  const int st = static_ws_address(&ws);
+  if (st) return st;
+  // Nothing in the scratch has to start at zero: the quantizer clears its own
+  // amax word on the stream before each use, and every other intermediate is
+  // written before it is read within the call.
+  return gdn_layer_fwd(w, cfg, x, y, S0, S_T, ws, (size_t)GDN_LAYER_STATIC_WS_BYTES, stream);
+}
