@@ -240,41 +240,15 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
     cp_async_wait_all();
     __syncthreads();
 
-    // ---------------------------------------------------- P0: gates
-    if (warp < 2) {
-      const int t = tid;
-      const float la = sm.lar[t];
-      float x = la;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (warp == 0 && lane == 31) sm.warp_tot = x;
-      sm.g2[t] = x;  // partial (warp-local) scan for now
-    }
-    __syncthreads();
-    if (tid < C) {
-      const float la = sm.lar[tid];
-      const float G = sm.g2[tid] + (tid >= 32 ? sm.warp_tot : 0.0f);
-      const float Gm1 = G - la;
-      sm.g2[tid] = G * kLog2e;
-      sm.g2m1[tid] = Gm1 * kLog2e;
-      const float bt = sm.ber[tid];
-      sm.be[tid] = bt;
-      sm.d1[tid] = bt * exp2f(Gm1 * kLog2e);
-      sm.eg[tid] = exp2f(G * kLog2e);
-    }
-    __syncthreads();
-    const float g2C = sm.g2[C - 1];
-    if (tid < C) sm.dk[tid] = exp2f(g2C - sm.g2[tid]);
-    // q, k: four threads per row (DK/4 columns each), FP32 norm, FP16 out
+    // ---------------------------------------------------- P0: gates, norms
+    // q, k rows: four threads per row (DK/4 columns each), FP32 norms.
+    constexpr int QC = DK / 4;
+    const int pr = tid >> 2, pq = tid & 3;
+    float qv[QC], kv[QC];
+    float nq, nk;
     {
-      constexpr int QC = DK / 4;
-      const int r = tid >> 2, qt = tid & 3;
-      const uint4* qsrc = reinterpret_cast<const uint4*>(&sm.qr[r * LDR + qt * QC]);
-      const uint4* ksrc = reinterpret_cast<const uint4*>(&sm.kr[r * LDR + qt * QC]);
-      float qv[QC], kv[QC];
+      const uint4* qsrc = reinterpret_cast<const uint4*>(&sm.qr[pr * LDR + pq * QC]);
+      const uint4* ksrc = reinterpret_cast<const uint4*>(&sm.kr[pr * LDR + pq * QC]);
       float qs = 0.f, ks = 0.f;
 #pragma unroll
       for (int i = 0; i < QC / 8; ++i) {
@@ -297,103 +271,137 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
       ks += __shfl_xor_sync(0xffffffffu, ks, 1);
       qs += __shfl_xor_sync(0xffffffffu, qs, 2);
       ks += __shfl_xor_sync(0xffffffffu, ks, 2);
-      const float nq = a.l2norm ? 1.0f / sqrtf(qs + 1e-6f) : 1.0f;
-      const float nk = a.l2norm ? 1.0f / sqrtf(ks + 1e-6f) : 1.0f;
-      __syncthreads();  // sm.dk visible
-      const float dkr = sm.dk[r] * nk;
+      nq = a.l2norm ? 1.0f / sqrtf(qs + 1e-6f) : 1.0f;
+      nk = a.l2norm ? 1.0f / sqrtf(ks + 1e-6f) : 1.0f;
+    }
+    // gates: warp 0, two tokens per lane, one inclusive scan of pair sums
+    if (warp == 0) {
+      const float la0 = sm.lar[2 * lane], la1 = sm.lar[2 * lane + 1];
+      const float pair = la0 + la1;
+      float x = pair;
 #pragma unroll
-      for (int i = 0; i < QC / 2; ++i) {
-        st_h2(&sm.qh[r * LDH + qt * QC + 2 * i], qv[2 * i] * nq, qv[2 * i + 1] * nq);
-        st_h2(&sm.kh[r * LDH + qt * QC + 2 * i], kv[2 * i] * nk, kv[2 * i + 1] * nk);
-        st_h2(&sm.kd[r * LDH + qt * QC + 2 * i], kv[2 * i] * dkr, kv[2 * i + 1] * dkr);
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const float ex = x - pair;                       // G before token 2*lane
+      const float G0 = ex + la0, G1 = x;
+      const float GC = __shfl_sync(0xffffffffu, x, 31);
+      const float b0 = sm.ber[2 * lane], b1 = sm.ber[2 * lane + 1];
+      const float Gs[2] = {G0, G1}, Gm[2] = {ex, G0}, bs[2] = {b0, b1};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * lane + e;
+        sm.g2[t] = Gs[e] * kLog2e;
+        sm.g2m1[t] = Gm[e] * kLog2e;
+        sm.be[t] = bs[e];
+        sm.d1[t] = bs[e] * exp2f(Gm[e] * kLog2e);
+        sm.eg[t] = exp2f(Gs[e] * kLog2e);
+        sm.dk[t] = exp2f((GC - Gs[e]) * kLog2e);
+      }
+      if (lane == 31) sm.warp_tot = GC * kLog2e;
+    }
+    __syncthreads();
+    const float g2C = sm.warp_tot;
+    {
+      const float dkr = sm.dk[pr] * nk;
+      uint4* qd = reinterpret_cast<uint4*>(&sm.qh[pr * LDH + pq * QC]);
+      uint4* kd = reinterpret_cast<uint4*>(&sm.kh[pr * LDH + pq * QC]);
+      uint4* dd = reinterpret_cast<uint4*>(&sm.kd[pr * LDH + pq * QC]);
+#pragma unroll
+      for (int i = 0; i < QC / 8; ++i) {
+        qd[i] = make_uint4(pack_h2(qv[8 * i] * nq, qv[8 * i + 1] * nq), pack_h2(qv[8 * i + 2] * nq, qv[8 * i + 3] * nq),
+                           pack_h2(qv[8 * i + 4] * nq, qv[8 * i + 5] * nq), pack_h2(qv[8 * i + 6] * nq, qv[8 * i + 7] * nq));
+        kd[i] = make_uint4(pack_h2(kv[8 * i] * nk, kv[8 * i + 1] * nk), pack_h2(kv[8 * i + 2] * nk, kv[8 * i + 3] * nk),
+                           pack_h2(kv[8 * i + 4] * nk, kv[8 * i + 5] * nk), pack_h2(kv[8 * i + 6] * nk, kv[8 * i + 7] * nk));
+        dd[i] = make_uint4(pack_h2(kv[8 * i] * dkr, kv[8 * i + 1] * dkr), pack_h2(kv[8 * i + 2] * dkr, kv[8 * i + 3] * dkr),
+                           pack_h2(kv[8 * i + 4] * dkr, kv[8 * i + 5] * dkr), pack_h2(kv[8 * i + 6] * dkr, kv[8 * i + 7] * dkr));
       }
     }
-    // beta o v as FP16
-    for (int i = tid; i < C * DVS / 2; i += NT) {
-      const int r = i / (DVS / 2), cc = (i % (DVS / 2)) * 2;
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(&sm.vr[r * LDV + cc]);
+    // beta o v as FP16, 8 columns per thread step
+    for (int i = tid; i < C * DVS / 8; i += NT) {
+      const int r = i / (DVS / 8), cc = (i % (DVS / 8)) * 8;
+      const uint4 w = *reinterpret_cast<const uint4*>(&sm.vr[r * LDV + cc]);
       const float bt = sm.be[r];
-      st_h2(&sm.vh[r * LDV + cc], bf16_bits_to_f32(w & 0xFFFFu) * bt, bf16_bits_to_f32(w >> 16) * bt);
+      *reinterpret_cast<uint4*>(&sm.vh[r * LDV + cc]) =
+          make_uint4(pack_h2(bf16_bits_to_f32(w.x & 0xFFFFu) * bt, bf16_bits_to_f32(w.x >> 16) * bt),
+                     pack_h2(bf16_bits_to_f32(w.y & 0xFFFFu) * bt, bf16_bits_to_f32(w.y >> 16) * bt),
+                     pack_h2(bf16_bits_to_f32(w.z & 0xFFFFu) * bt, bf16_bits_to_f32(w.z >> 16) * bt),
+                     pack_h2(bf16_bits_to_f32(w.w & 0xFFFFu) * bt, bf16_bits_to_f32(w.w >> 16) * bt));
     }
     __syncthreads();
     // staging is free: prefetch the next chunk
     if (ch + 1 < nchunks)
       issue_chunk_loads<DK, DVS>(sm, a, tok0 + t0 + C, h, dv_off, (int)(T - t0 - C < C ? T - t0 - C : C), tid);
 
-    // ---------------------------------------------------- P1: K K^T, Q K^T
-    {
-      // warps 0-3: K K^T -> L ; warps 4-7: Q K^T -> A.  Row tile mrow, column
-      // tiles 0 .. 2*mrow+1 (the causal part).
-      const __half* Ab = nhalf == 0 ? sm.kh : sm.qh;
-      float acc[8][4];
+    // ---------------------------------------------------- P1: K K^T -> L
+    // The ten lower-triangular 16x16 blocks (i, j <= i), one or two per warp.
+#pragma unroll 1
+    for (int task = warp; task < 10; task += 8) {
+      const int bi = task < 1 ? 0 : task < 3 ? 1 : task < 6 ? 2 : 3;
+      const int bj = task - bi * (bi + 1) / 2;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < DK / 16; ++kk) {
-        uint32_t af[4];
-        frag_a(af, Ab, LDH, 16 * mrow, 16 * kk, lane);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          if (jj <= mrow) {
-            uint32_t bf[4];
-            frag_b_nk(bf, sm.kh, LDH, 16 * kk, 16 * jj, lane);
-            mma16816(acc[2 * jj], af, bf[0], bf[1]);
-            mma16816(acc[2 * jj + 1], af, bf[2], bf[3]);
-          }
-        }
+      for (int kk = 0; kk < DK / 16; kk += 2) {   // two k-chains in flight
+        uint32_t af[4], bf[4], af2[4], bf2[4];
+        frag_a(af, sm.kh, LDH, 16 * bi, 16 * kk, lane);
+        frag_b_nk(bf, sm.kh, LDH, 16 * kk, 16 * bj, lane);
+        frag_a(af2, sm.kh, LDH, 16 * bi, 16 * kk + 16, lane);
+        frag_b_nk(bf2, sm.kh, LDH, 16 * kk + 16, 16 * bj, lane);
+        mma16816(acc[0], af, bf[0], bf[1]);
+        mma16816(acc[1], af, bf[2], bf[3]);
+        mma16816(acc2[0], af2, bf2[0], bf2[1]);
+        mma16816(acc2[1], af2, bf2[2], bf2[3]);
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j <= 2 * mrow + 1) {
+      for (int n = 0; n < 2; ++n)
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int t = 16 * mrow + g + hh * 8;
-            const int s0 = 8 * j + 2 * c4;
-            float v0, v1;
-            if (nhalf == 0) {
-              const float bt = sm.be[t], gm = sm.g2m1[t];
-              v0 = (s0 < t) ? bt * exp2f(gm - sm.g2[s0]) * acc[j][2 * hh] : 0.f;
-              v1 = (s0 + 1 < t) ? bt * exp2f(gm - sm.g2[s0 + 1]) * acc[j][2 * hh + 1] : 0.f;
-              st_h2(&sm.lh[t * LDX + s0], v0, v1);
-            } else {
-              const float gt = sm.g2[t];
-              v0 = (s0 <= t) ? exp2f(gt - sm.g2[s0]) * acc[j][2 * hh] : 0.f;
-              v1 = (s0 + 1 <= t) ? exp2f(gt - sm.g2[s0 + 1]) * acc[j][2 * hh + 1] : 0.f;
-              st_h2(&sm.ah[t * LDX + s0], v0, v1);
-            }
-          }
+        for (int e = 0; e < 4; ++e) acc[n][e] += acc2[n][e];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int t = 16 * bi + g + hh * 8;
+          const int s0 = 16 * bj + 8 * n + 2 * c4;
+          const float bt = sm.be[t], gm = sm.g2m1[t];
+          const float v0 = (s0 < t) ? bt * exp2f(gm - sm.g2[s0]) * acc[n][2 * hh] : 0.f;
+          const float v1 = (s0 + 1 < t) ? bt * exp2f(gm - sm.g2[s0 + 1]) * acc[n][2 * hh + 1] : 0.f;
+          st_h2(&sm.lh[t * LDX + s0], v0, v1);
         }
-      }
     }
     __syncthreads();
 
-    // ---------------------------------------------------- P2: X = (I+L)^-1
-    if (warp < 4 && lane < 16) {
-      // diagonal block `warp`, column j = lane, forward substitution
-      const int base = 16 * warp;
-      const int j = lane;
-      float x[16];
+    // ------------------------------- P2: X = (I+L)^-1 (warps 0-3) || Q K^T (warps 4-7)
+    if (warp < 4) {
+      if (lane < 16) {
+        // diagonal block `warp`, column j = lane, forward substitution in FP32
+        const int base = 16 * warp;
+        const int j = lane;
+        float lrow[16][16];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        float acc = (t == j) ? 1.0f : 0.0f;
+        for (int t = 1; t < 16; ++t)
 #pragma unroll
-        for (int s = 0; s < t; ++s) acc -= __half2float(sm.lh[(base + t) * LDX + base + s]) * x[s];
-        x[t] = (t < j) ? 0.0f : acc;
+          for (int s2 = 0; s2 < t; ++s2) lrow[t][s2] = __half2float(sm.lh[(base + t) * LDX + base + s2]);
+        float x[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          float acc = (t == j) ? 1.0f : 0.0f;
+#pragma unroll
+          for (int s2 = 0; s2 < t; ++s2) acc -= lrow[t][s2] * x[s2];
+          x[t] = (t < j) ? 0.0f : acc;
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) sm.xh[(base + t) * LDX + base + j] = __float2half_rn(x[t]);
       }
-#pragma unroll
-      for (int t = 0; t < 16; ++t) sm.xh[(base + t) * LDX + base + j] = __float2half_rn(x[t]);
-    }
-    __syncthreads();
-    {
-      // off-diagonal blocks, one level (distance) at a time; warp i (< 4)
-      // owns block row i and keeps P_ik = X_ii L_ik in registers.
-      uint32_t P[3][4];  // P[i-1-k'] for k = i-1, i-2, i-3
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // off-diagonal blocks, one level (distance) at a time; warp i owns block
+      // row i and keeps P_ik = X_ii L_ik in registers.
+      uint32_t P[3][4];
+#pragma unroll 1
       for (int d = 1; d < 4; ++d) {
-        if (warp < 4 && warp >= d) {
+        if (warp >= d) {
           const int i = warp, jb = warp - d;
-          // new P for k = i - d: X_ii * L_{i,i-d}
           {
             float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t af[4], bf[4];
@@ -403,7 +411,6 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
             mma16816(p1, af, bf[2], bf[3]);
             c_to_a(P[d - 1], p0, p1);
           }
-          // X_{i,jb} = - sum_{k=jb}^{i-1} P_ik X_{k,jb}
           float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int dd = 1; dd <= 3; ++dd) {
@@ -422,9 +429,46 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
           st_h2(&sm.xh[r0 * LDX + cc + 8], -z1[0], -z1[1]);
           st_h2(&sm.xh[(r0 + 8) * LDX + cc + 8], -z1[2], -z1[3]);
         }
-        __syncthreads();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+    } else {
+      // Gamma o Q K^T: the ten lower blocks over warps 4-7
+#pragma unroll 1
+      for (int task = warp - 4; task < 10; task += 4) {
+        const int bi = task < 1 ? 0 : task < 3 ? 1 : task < 6 ? 2 : 3;
+        const int bj = task - bi * (bi + 1) / 2;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; kk += 2) {
+          uint32_t af[4], bf[4], af2[4], bf2[4];
+          frag_a(af, sm.qh, LDH, 16 * bi, 16 * kk, lane);
+          frag_b_nk(bf, sm.kh, LDH, 16 * kk, 16 * bj, lane);
+          frag_a(af2, sm.qh, LDH, 16 * bi, 16 * kk + 16, lane);
+          frag_b_nk(bf2, sm.kh, LDH, 16 * kk + 16, 16 * bj, lane);
+          mma16816(acc[0], af, bf[0], bf[1]);
+          mma16816(acc[1], af, bf[2], bf[3]);
+          mma16816(acc2[0], af2, bf2[0], bf2[1]);
+          mma16816(acc2[1], af2, bf2[2], bf2[3]);
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[n][e] += acc2[n][e];
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int t = 16 * bi + g + hh * 8;
+            const int s0 = 16 * bj + 8 * n + 2 * c4;
+            const float gt = sm.g2[t];
+            const float v0 = (s0 <= t) ? exp2f(gt - sm.g2[s0]) * acc[n][2 * hh] : 0.f;
+            const float v1 = (s0 + 1 <= t) ? exp2f(gt - sm.g2[s0 + 1]) * acc[n][2 * hh + 1] : 0.f;
+            st_h2(&sm.ah[t * LDX + s0], v0, v1);
+          }
       }
     }
+    __syncthreads();
     // X diag(d1): lower blocks only
     for (int i = tid; i < C * C / 2; i += NT) {
       const int r = i / (C / 2), cc = (i % (C / 2)) * 2;
@@ -502,18 +546,49 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
       for (int j = 0; j < NVH; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) OQ[j][e] = 0.f;
+      constexpr int NP = (NVH % 2 != 0) ? 4 : 1;
+      float Up[NP][NVH][4], OQp[NP][NVH][4];
+#pragma unroll
+      for (int q = 0; q < NP; ++q)
+#pragma unroll
+        for (int j = 0; j < NVH; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) Up[q][j][e] = OQp[q][j][e] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < DK / 16; ++kk) {
         uint32_t aw[4], aq[4];
         frag_a(aw, sm.wh, LDH, 16 * mrow, 16 * kk, lane);
         frag_a(aq, sm.qh, LDH, 16 * mrow, 16 * kk, lane);
+        if constexpr (NVH % 2 == 0) {
 #pragma unroll
-        for (int j = 0; j < NVH; ++j) {
-          uint32_t b0, b1;
-          frag_b_kn1(b0, b1, sm.sh, LDV, 16 * kk, 8 * (nhalf * NVH + j), lane);
-          mma16816(U[j], aw, b0, b1);
-          mma16816(OQ[j], aq, b0, b1);
+          for (int j = 0; j < NVH; j += 2) {
+            uint32_t bf[4];
+            frag_b_kn(bf, sm.sh, LDV, 16 * kk, 8 * (nhalf * NVH + j), lane);
+            mma16816(U[j], aw, bf[0], bf[1]);
+            mma16816(OQ[j], aq, bf[0], bf[1]);
+            mma16816(U[j + 1], aw, bf[2], bf[3]);
+            mma16816(OQ[j + 1], aq, bf[2], bf[3]);
+          }
+        } else {
+          // one n-tile per warp: the k-loop is the only parallelism, so four
+          // partial sums keep four MMA chains in flight
+#pragma unroll
+          for (int j = 0; j < NVH; ++j) {
+            uint32_t b0, b1;
+            frag_b_kn1(b0, b1, sm.sh, LDV, 16 * kk, 8 * (nhalf * NVH + j), lane);
+            mma16816(Up[kk & 3][j], aw, b0, b1);
+            mma16816(OQp[kk & 3][j], aq, b0, b1);
+          }
         }
+      }
+      if constexpr (NVH % 2 != 0) {
+#pragma unroll
+        for (int j = 0; j < NVH; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            U[j][e] += (Up[0][j][e] + Up[1][j][e]) + (Up[2][j][e] + Up[3][j][e]);
+            OQ[j][e] = (OQp[0][j][e] + OQp[1][j][e]) + (OQp[2][j][e] + OQp[3][j][e]);
+          }
       }
     }
     // U (the new values) -> FP16, replacing beta o v
@@ -539,11 +614,21 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
         if (kk <= mrow) {
           uint32_t af[4];
           frag_a(af, sm.ah, LDX, 16 * mrow, 16 * kk, lane);
+          if constexpr (NVH % 2 == 0) {
 #pragma unroll
-          for (int j = 0; j < NVH; ++j) {
-            uint32_t b0, b1;
-            frag_b_kn1(b0, b1, sm.vh, LDV, 16 * kk, 8 * (nhalf * NVH + j), lane);
-            mma16816(OQ[j], af, b0, b1);
+            for (int j = 0; j < NVH; j += 2) {
+              uint32_t bf[4];
+              frag_b_kn(bf, sm.vh, LDV, 16 * kk, 8 * (nhalf * NVH + j), lane);
+              mma16816(OQ[j], af, bf[0], bf[1]);
+              mma16816(OQ[j + 1], af, bf[2], bf[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < NVH; ++j) {
+              uint32_t b0, b1;
+              frag_b_kn1(b0, b1, sm.vh, LDV, 16 * kk, 8 * (nhalf * NVH + j), lane);
+              mma16816(OQ[j], af, b0, b1);
+            }
           }
         }
       }
@@ -573,16 +658,46 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
       for (int j = 0; j < NVT; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) S[j][e] *= eC;
+      if constexpr (NVT <= 4) {
+        // few n-tiles: two k-chains in flight, summed into S at the end
+        float S2[NVT][4];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t af[4];
-        frag_a_t(af, sm.kd, LDH, 16 * warp, 16 * kk, lane);
+        for (int j = 0; j < NVT; ++j)
 #pragma unroll
-        for (int j = 0; j < NVT; j += 2) {
-          uint32_t bf[4];
-          frag_b_kn(bf, sm.vh, LDV, 16 * kk, 8 * j, lane);
-          mma16816(S[j], af, bf[0], bf[1]);
-          mma16816(S[j + 1], af, bf[2], bf[3]);
+          for (int e = 0; e < 4; ++e) S2[j][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t af[4];
+          frag_a_t(af, sm.kd, LDH, 16 * warp, 16 * kk, lane);
+#pragma unroll
+          for (int j = 0; j < NVT; j += 2) {
+            uint32_t bf[4];
+            frag_b_kn(bf, sm.vh, LDV, 16 * kk, 8 * j, lane);
+            if (kk & 1) {
+              mma16816(S2[j], af, bf[0], bf[1]);
+              mma16816(S2[j + 1], af, bf[2], bf[3]);
+            } else {
+              mma16816(S[j], af, bf[0], bf[1]);
+              mma16816(S[j + 1], af, bf[2], bf[3]);
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < NVT; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) S[j][e] += S2[j][e];
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t af[4];
+          frag_a_t(af, sm.kd, LDH, 16 * warp, 16 * kk, lane);
+#pragma unroll
+          for (int j = 0; j < NVT; j += 2) {
+            uint32_t bf[4];
+            frag_b_kn(bf, sm.vh, LDV, 16 * kk, 8 * j, lane);
+            mma16816(S[j], af, bf[0], bf[1]);
+            mma16816(S[j + 1], af, bf[2], bf[3]);
+          }
         }
       }
     }
