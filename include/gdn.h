@@ -86,6 +86,9 @@ int gdn_stream_check(gdn_stream_t stream);
  *                      g_enc  = 2688 / amax_t (1 if amax_t == 0; FLT_MAX if
  *                      the quotient overflows);
  *   GIVEN_SCALE mode:  g_enc  = *g_enc_in (device scalar, > 0, finite).
+ *   GIVEN_AMAX mode:   amax_t = *g_enc_in (device scalar: the tensor's amax,
+ *                      e.g. recorded by the kernel that produced x), then as
+ *                      DYNAMIC without the amax pass.
  *   per 16-block:      s = E4M3_satfinite((amax_b / 6) * g_enc);
  *                      code_i = E2M1_satfinite(x_i * (g_enc / s))
  *                      (all codes 0 when s == 0; a negative value that rounds
@@ -104,10 +107,10 @@ int gdn_stream_check(gdn_stream_t stream);
  * g_out    device float, written with the decode scale.
  * ws       DYNAMIC mode only: gdn_quantize_workspace_size() bytes, 16-byte
  *          aligned (holds the running amax; overwritten).  May be NULL in
- *          GIVEN_SCALE mode.
+ *          the GIVEN_* modes.
  * rows == 0 is valid (only *g_out is written).
  * ------------------------------------------------------------------------ */
-enum { GDN_QUANT_DYNAMIC = 0, GDN_QUANT_GIVEN_SCALE = 1 };
+enum { GDN_QUANT_DYNAMIC = 0, GDN_QUANT_GIVEN_SCALE = 1, GDN_QUANT_GIVEN_AMAX = 2 };
 enum { GDN_DTYPE_BF16 = 0, GDN_DTYPE_F32 = 1 };
 enum { GDN_SF_TILED = 0, GDN_SF_LINEAR = 1 };
 

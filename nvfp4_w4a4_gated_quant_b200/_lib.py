@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgdn.so")
 
 GDN_OK = 0
-QUANT_DYNAMIC, QUANT_GIVEN_SCALE = 0, 1
+QUANT_DYNAMIC, QUANT_GIVEN_SCALE, QUANT_GIVEN_AMAX = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SF_TILED, SF_LINEAR = 0, 1
 EPI_STORE_BF16, EPI_STORE_F32, EPI_LOG_ALPHA, EPI_BETA = 0, 1, 2, 3
@@ -141,12 +141,13 @@ def scales_tiled_bytes(rows, cols):
 
 
 def gdn_quantize_nvfp4(x, g_enc=None, layout="tiled", codes=None, scales=None, sf_row_offset=0, g_out=None,
-                       ws=None, stream=None):
+                       ws=None, stream=None, amax=None):
     """Quantize a 2-D bf16 / FP32 CUDA tensor (unit stride along columns).
 
     Dynamic per-tensor scale unless ``g_enc`` (a 1-element FP32 CUDA tensor
-    holding the encode scale) is given.  Returns (codes, scales, g) where g is
-    the 1-element FP32 decode scale.  ``scales`` may be a shared TILED buffer
+    holding the encode scale) or ``amax`` (a 1-element FP32 CUDA tensor holding
+    the tensor's amax) is given.  Returns (codes, scales, g) where g is the
+    1-element FP32 decode scale.  ``scales`` may be a shared TILED buffer
     filled from row ``sf_row_offset`` on."""
     if x.dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("x must be bf16 or float32")
@@ -166,9 +167,14 @@ def gdn_quantize_nvfp4(x, g_enc=None, layout="tiled", codes=None, scales=None, s
     _need(scales, torch.uint8, "scales", dev)
     _need(g_out, torch.float32, "g_out", dev)
     mode = QUANT_DYNAMIC
+    if g_enc is not None and amax is not None:
+        raise ValueError("give g_enc or amax, not both")
     if g_enc is not None:
         _need(g_enc, torch.float32, "g_enc", dev)
         mode = QUANT_GIVEN_SCALE
+    if amax is not None:
+        _need(amax, torch.float32, "amax", dev)
+        g_enc, mode = amax, QUANT_GIVEN_AMAX
     L = lib()
     wsz = int(L.gdn_quantize_workspace_size())
     if ws is None and mode == QUANT_DYNAMIC:

@@ -79,10 +79,11 @@ int check_quant_args(const void* x, int x_dtype, int64_t rows, int64_t cols, int
   if (rows < 0 || cols <= 0 || ld_x < cols || !g_out) return GDN_ERR_INVALID_ARG;
   if (x_dtype != GDN_DTYPE_BF16 && x_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARG;
   const int64_t per16 = x_dtype == GDN_DTYPE_F32 ? 4 : 8;  // elements per 16 bytes
-  if (mode != GDN_QUANT_DYNAMIC && mode != GDN_QUANT_GIVEN_SCALE) return GDN_ERR_INVALID_ARG;
+  if (mode != GDN_QUANT_DYNAMIC && mode != GDN_QUANT_GIVEN_SCALE && mode != GDN_QUANT_GIVEN_AMAX)
+    return GDN_ERR_INVALID_ARG;
   if (sf_layout != GDN_SF_TILED && sf_layout != GDN_SF_LINEAR) return GDN_ERR_INVALID_ARG;
   if (sf_row_offset < 0 || (sf_layout == GDN_SF_LINEAR && sf_row_offset != 0)) return GDN_ERR_INVALID_ARG;
-  if (mode == GDN_QUANT_GIVEN_SCALE && !g_enc_in) return GDN_ERR_INVALID_ARG;
+  if (mode != GDN_QUANT_DYNAMIC && !g_enc_in) return GDN_ERR_INVALID_ARG;
   if (mode == GDN_QUANT_DYNAMIC && (!ws || ws_bytes < kQuantWs)) return GDN_ERR_WORKSPACE;
   if (cols % 16 != 0 || (sf_layout == GDN_SF_TILED && cols % 64 != 0)) return GDN_ERR_UNSUPPORTED_SHAPE;
   if (rows > 0 && (!x || !codes || !scales)) return GDN_ERR_INVALID_ARG;
@@ -208,7 +209,7 @@ int gdn_delta_rule_fwd(const void* q, const void* k, const void* v, int64_t ld_q
   if ((S0 && !aligned(S0, 4)) || (S_T && !aligned(S_T, 4))) return GDN_ERR_ALIGNMENT;
   return launch_delta_rule(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
                            static_cast<const uint16_t*>(v), ld_q, ld_k, ld_v, log_alpha, beta, S0, B, T, H, dk, dv,
-                           flags, o, S_T, as_stream(stream));
+                           flags, o, S_T, nullptr, as_stream(stream));
 }
 
 }  // extern "C"

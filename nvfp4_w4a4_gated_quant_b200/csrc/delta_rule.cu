@@ -163,6 +163,7 @@ struct Args {
   int l2norm;
   void* o;
   float* S_T;
+  unsigned* o_amax;   // optional: FP32 bits of max |stored o| (atomicMax), for the next quantizer
 };
 
 template <int DK, int DVS>
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
       S[j][e] = (a.S0 && s_owner) ? a.S0[((int64_t)chain * DK + r) * a.dv + dv_off + col] : 0.0f;
     }
 
+  uint32_t amax_bits = 0;   // FP32 bits of the largest |o| this thread stored
   const int64_t nchunks = (T + C - 1) / C;
   if (nchunks > 0) issue_chunk_loads<DK, DVS>(sm, a, tok0, h, dv_off, (int)(T < C ? T : C), tid);
 
@@ -643,9 +645,12 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
             if (O_F32) {
               *reinterpret_cast<float2*>(reinterpret_cast<float*>(a.o) + orow + cc) =
                   make_float2(OQ[j][2 * hh], OQ[j][2 * hh + 1]);
+              amax_bits = max(amax_bits, max(__float_as_uint(OQ[j][2 * hh]) & 0x7FFFFFFFu,
+                                             __float_as_uint(OQ[j][2 * hh + 1]) & 0x7FFFFFFFu));
             } else {
-              *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(a.o) + orow + cc) =
-                  f32_to_bf16_bits(OQ[j][2 * hh]) | (f32_to_bf16_bits(OQ[j][2 * hh + 1]) << 16);
+              const uint32_t b0 = f32_to_bf16_bits(OQ[j][2 * hh]), b1 = f32_to_bf16_bits(OQ[j][2 * hh + 1]);
+              *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(a.o) + orow + cc) = b0 | (b1 << 16);
+              amax_bits = max(amax_bits, max(b0 & 0x7FFFu, b1 & 0x7FFFu) << 16);
             }
           }
         }
@@ -704,6 +709,11 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
     __syncthreads();
   }
 
+  if (a.o_amax) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
+    if (lane == 0 && amax_bits) atomicMax(a.o_amax, amax_bits);
+  }
   if (a.S_T && s_owner) {
 #pragma unroll
     for (int j = 0; j < NVT; ++j)
@@ -739,7 +749,8 @@ int launch_dk(const Args& a, int dvs, int64_t chains, cudaStream_t stream) {
 
 int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                       int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
-                      int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, cudaStream_t stream) {
+                      int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
+                      cudaStream_t stream) {
   const int64_t chains = B * H;
   if (chains == 0) return GDN_OK;
   // Split d_v so that the CTAs cover the SMs (one CTA per SM).
@@ -763,6 +774,7 @@ int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
   a.l2norm = (flags & GDN_DR_L2NORM_QK) ? 1 : 0;
   a.o = o;
   a.S_T = S_T;
+  a.o_amax = o_amax;
   const bool f32 = (flags & GDN_DR_O_FP32) != 0;
   switch (dk) {
     case 32: return f32 ? launch_dk<32, true>(a, dvs, chains, stream) : launch_dk<32, false>(a, dvs, chains, stream);

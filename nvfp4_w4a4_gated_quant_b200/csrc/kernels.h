@@ -21,6 +21,7 @@ int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t*
 
 int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                       int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
-                      int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, cudaStream_t stream);
+                      int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
+                      cudaStream_t stream);
 
 }  // namespace gdn

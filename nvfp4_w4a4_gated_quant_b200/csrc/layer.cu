@@ -94,7 +94,6 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
   uint8_t* o_scales = base + off[GDN_WS_O_SCALES];
   float* o_g = reinterpret_cast<float*>(base + off[GDN_WS_O_G]);
   void* qws = base + off[GDN_WS_QUANT];
-  void* sws = base + off[GDN_WS_SCAN];
   const size_t qws_bytes = gdn_quantize_workspace_size();
   gdn_stream_t s = stream;
 
@@ -112,12 +111,17 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
   st = gdn_gemm_nvfp4(&xa, x_g, &w->w_qkvab, M, NQKV + 2 * H, D, seg, 5, s);
   if (st) return st;
 
-  st = gdn_delta_rule_fwd(qkv, qkv + HK, qkv + 2 * HK, NQKV, NQKV, NQKV, log_alpha, beta, S0, cfg->B, cfg->T, H, dk, dv,
-                          GDN_DR_L2NORM_QK, o, S_T, sws, 0, s);
+  // The scan records max |o| of the bf16 values it stores, so o is
+  // quantized in one pass (given-amax mode) instead of amax pass + pass.
+  unsigned* o_amax = static_cast<unsigned*>(qws);
+  cudaError_t ce = cudaMemsetAsync(o_amax, 0, sizeof(unsigned), reinterpret_cast<cudaStream_t>(s));
+  if (ce != cudaSuccess) return record_cuda_error(ce);
+  st = launch_delta_rule(qkv, qkv + HK, qkv + 2 * HK, NQKV, NQKV, NQKV, log_alpha, beta, S0, cfg->B, cfg->T, H, dk, dv,
+                         GDN_DR_L2NORM_QK, o, S_T, o_amax, reinterpret_cast<cudaStream_t>(s));
   if (st) return st;
 
-  st = gdn_quantize_nvfp4(o, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_DYNAMIC, nullptr, o_codes, o_scales, GDN_SF_TILED, 0, o_g, qws,
-                          qws_bytes, s);
+  st = gdn_quantize_nvfp4(o, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_GIVEN_AMAX, reinterpret_cast<const float*>(o_amax),
+                          o_codes, o_scales, GDN_SF_TILED, 0, o_g, nullptr, 0, s);
   if (st) return st;
 
   gdn_nvfp4_t oa{o_codes, o_scales};

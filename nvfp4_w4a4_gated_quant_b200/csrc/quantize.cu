@@ -112,51 +112,68 @@ __device__ __forceinline__ uint32_t e2m1x8(const float* r) {
   return out;
 }
 
+// Byte offset of the scale of (row R, 16-element group j) in the tiled layout.
+__device__ __forceinline__ int64_t scale_offset(int64_t R, int64_t j, int64_t kc) {
+  return (R >> 7) * kc * 512 + (j >> 2) * 512 + (R & 31) * 16 + ((R & 127) >> 5) * 4 + (j & 3);
+}
+
+// One 16-element block: E4M3 scale, eight packed code bytes, one scale byte.
+template <typename In>
+__device__ __forceinline__ void quant_block(const uint4 (&v)[16 / In::kPerVec], float g_enc, uint8_t* codes,
+                                            uint8_t* scale) {
+  constexpr int NV = 16 / In::kPerVec;
+  uint32_t mb = 0;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) mb = max(mb, In::absmax_bits(v[i]));
+  const float amax_b = __uint_as_float(mb);
+  const float s_f = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g_enc);
+  const uint32_t s = e4m3_satfinite(s_f);
+  const float s_val = e4m3_value(s);
+  uint2 packed = make_uint2(0u, 0u);
+  if (s_val > 0.0f) {
+    const float inv = __fdiv_rn(g_enc, s_val);
+    float rr[16];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) In::to_f32(v[i], rr + i * In::kPerVec);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) rr[i] = __fmul_rn(rr[i], inv);
+    packed.x = e2m1x8(rr);
+    packed.y = e2m1x8(rr + 8);
+  }
+  *reinterpret_cast<uint2*>(codes) = packed;
+  *scale = (uint8_t)s;
+}
+
 template <typename In, typename E>
 __global__ void quant_kernel(const E* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                              int mode, const float* __restrict__ g_enc_in,
                              const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes,
                              uint8_t* __restrict__ scales, int tiled, int64_t row_off,
                              float* __restrict__ g_out) {
-  const float g_enc = (mode == GDN_QUANT_DYNAMIC) ? encode_scale_from_amax(__uint_as_float(*amax_bits))
-                                                  : *g_enc_in;
+  const float g_enc = mode == GDN_QUANT_DYNAMIC      ? encode_scale_from_amax(__uint_as_float(*amax_bits))
+                      : mode == GDN_QUANT_GIVEN_AMAX ? encode_scale_from_amax(*g_enc_in)
+                                                     : *g_enc_in;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *g_out = __fdiv_rn(1.0f, g_enc);
   const int64_t bpr = cols >> 4;  // 16-element blocks per row
   const int64_t kc = cols >> 6;   // 64-element scale chunks per row (TILED)
-  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
-    const E* row = x + r * ld;
+  // Two rows per step so that each thread has two blocks' loads in flight.
+  for (int64_t r = blockIdx.y; r < rows; r += 2 * (int64_t)gridDim.y) {
+    const int64_t r2 = r + gridDim.y;
+    const bool two = r2 < rows;
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < bpr; j += (int64_t)gridDim.x * blockDim.x) {
       constexpr int NV = 16 / In::kPerVec;
-      uint4 vv[NV];
-      uint32_t mb = 0;
+      uint4 va[NV], vb[NV];
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        vv[i] = ld_vec(row + j * 16 + i * In::kPerVec);
-        mb = max(mb, In::absmax_bits(vv[i]));
-      }
-      const float amax_b = __uint_as_float(mb);
-      const float s_f = __fmul_rn(__fdiv_rn(amax_b, 6.0f), g_enc);
-      const uint32_t s = e4m3_satfinite(s_f);
-      const float s_val = e4m3_value(s);
-      uint2 packed = make_uint2(0u, 0u);
-      if (s_val > 0.0f) {
-        const float inv = __fdiv_rn(g_enc, s_val);
-        float rr[16];
+      for (int i = 0; i < NV; ++i) va[i] = ld_vec(x + r * ld + j * 16 + i * In::kPerVec);
+      if (two) {
 #pragma unroll
-        for (int i = 0; i < NV; ++i) In::to_f32(vv[i], rr + i * In::kPerVec);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) rr[i] = __fmul_rn(rr[i], inv);
-        packed.x = e2m1x8(rr);
-        packed.y = e2m1x8(rr + 8);
+        for (int i = 0; i < NV; ++i) vb[i] = ld_vec(x + r2 * ld + j * 16 + i * In::kPerVec);
       }
-      *reinterpret_cast<uint2*>(codes + r * (cols >> 1) + j * 8) = packed;
-      if (tiled) {
-        const int64_t R = r + row_off;
-        const int64_t off = (R >> 7) * kc * 512 + (j >> 2) * 512 + (R & 31) * 16 + ((R & 127) >> 5) * 4 + (j & 3);
-        scales[off] = (uint8_t)s;
-      } else {
-        scales[r * bpr + j] = (uint8_t)s;
-      }
+      quant_block<In>(va, g_enc, codes + r * (cols >> 1) + j * 8,
+                      tiled ? scales + scale_offset(r + row_off, j, kc) : scales + r * bpr + j);
+      if (two)
+        quant_block<In>(vb, g_enc, codes + r2 * (cols >> 1) + j * 8,
+                        tiled ? scales + scale_offset(r2 + row_off, j, kc) : scales + r2 * bpr + j);
     }
   }
 }

@@ -46,6 +46,20 @@ def test_quantize_linear_layout_and_given_scale():
     _check_quant(x, xd, g_enc=np.float32(37.5))
 
 
+def test_quantize_given_amax_equals_dynamic():
+    """Given-amax mode (the amax recorded by the producer of the tensor) gives
+    the dynamic result without the amax pass."""
+    x = inputs.activations(np.random.default_rng(12), (257, 320))
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    amax = torch.tensor([float(np.abs(x).max())], dtype=torch.float32, device="cuda")
+    c1, s1, g1 = _lib.gdn_quantize_nvfp4(xd)
+    c2, s2, g2 = _lib.gdn_quantize_nvfp4(xd, amax=amax)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(s1, s2) and torch.equal(g1, g2)
+    ref = nvfp4.quantize(x)
+    np.testing.assert_array_equal(to_np(c2), ref["codes"])
+
+
 def test_quantize_fp32_weights_bit_exact():
     w = inputs.weight(np.random.default_rng(6), 200, 256)
     _check_quant(w, f32_cuda(w))
