@@ -73,6 +73,12 @@ const char* gdn_version(void);
  * (GDN_OK, or GDN_ERR_TIMEOUT when a bounded device wait ran out), or
  * GDN_ERR_CUDA when the synchronisation itself failed. */
 int gdn_stream_check(gdn_stream_t stream);
+/* Diagnostic: enqueue a one-warp kernel that waits, at most poll_limit polls
+ * (1 .. 2^26), on an mbarrier nothing arrives on -- the bounded wait the
+ * pipelined kernels use -- and so records GDN_ERR_TIMEOUT in the device
+ * status word; gdn_stream_check() then returns and clears it.  Checks the
+ * watchdog path without faulting or hanging anything. */
+int gdn_selftest_bounded_wait(uint32_t poll_limit, gdn_stream_t stream);
 
 /* ------------------------------------------------------------------------ *
  * Step 1: quantize activations to NVFP4.

@@ -66,6 +66,7 @@ def lib():
             "gdn_last_error": (ctypes.c_char_p, []),
             "gdn_version": (ctypes.c_char_p, []),
             "gdn_stream_check": (ctypes.c_int, [c_vp]),
+            "gdn_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, c_vp]),
             "gdn_quantize_workspace_size": (ctypes.c_size_t, []),
             "gdn_scales_tiled_bytes": (ctypes.c_size_t, [c_i64, c_i64]),
             "gdn_quantize_nvfp4": (ctypes.c_int, [c_vp, ctypes.c_int, c_i64, c_i64, c_i64, ctypes.c_int, c_vp,
@@ -94,7 +95,7 @@ def lib():
     return _LIB
 
 
-EXPORTED = ("gdn_status_string", "gdn_last_error", "gdn_version", "gdn_stream_check",
+EXPORTED = ("gdn_status_string", "gdn_last_error", "gdn_version", "gdn_stream_check", "gdn_selftest_bounded_wait",
             "gdn_quantize_workspace_size", "gdn_scales_tiled_bytes", "gdn_quantize_nvfp4", "gdn_gemm_nvfp4",
             "gdn_gates", "gdn_delta_rule_workspace_size", "gdn_delta_rule_fwd", "gdn_layer_workspace_size",
             "gdn_layer_workspace_offsets", "gdn_layer_fwd", "gdn_layer_fwd_static_ws")

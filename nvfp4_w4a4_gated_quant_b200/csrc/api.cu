@@ -14,6 +14,26 @@ namespace gdn {
 namespace {
 __device__ int g_status_word = GDN_OK;
 
+// Waits on an mbarrier that nothing ever arrives on, with the same bounded
+// poll-and-back-off loop the pipelined kernels use, then reports
+// GDN_ERR_TIMEOUT through the device status word and returns.
+__global__ void bounded_wait_selftest_kernel(uint32_t poll_limit, int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool done = false;
+    for (uint32_t i = 0; i < poll_limit && !done; ++i) {
+      done = mbar_try_wait(&bar, 0);
+      if (!done) __nanosleep(32);
+    }
+    if (!done) report_status(status, GDN_ERR_TIMEOUT);
+  }
+}
+
 thread_local char t_last_error[256] = "no error";
 
 constexpr int kMaxDevices = 64;
@@ -71,6 +91,8 @@ using namespace gdn;
 namespace {
 constexpr size_t kQuantWs = 256;
 
+
+
 cudaStream_t as_stream(gdn_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int check_quant_args(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, int mode, const float* g_enc_in,
@@ -127,6 +149,14 @@ int gdn_stream_check(gdn_stream_t stream) {
     if (e != cudaSuccess) return record_cuda_error(e);
   }
   return word;
+}
+
+int gdn_selftest_bounded_wait(uint32_t poll_limit, gdn_stream_t stream) {
+  if (poll_limit == 0 || poll_limit > (1u << 26)) return GDN_ERR_INVALID_ARG;
+  int* status = device_status_word();
+  if (!status) return record_cuda_error(cudaErrorInvalidDevice);
+  gdn::bounded_wait_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(poll_limit, status);
+  return check_launch();
 }
 
 size_t gdn_quantize_workspace_size(void) { return kQuantWs; }

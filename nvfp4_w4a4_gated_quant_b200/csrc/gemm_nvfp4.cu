@@ -8,7 +8,10 @@
 // segment (section "Critical Lessons for Model Serving": modules scaled
 // separately must not share one global scale inside a fused kernel).
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles, M fastest):
+// Design (one CTA per SM, persistent over 128 x 256 output tiles, N fastest:
+// the CTAs in flight share a few 128-row blocks of A and sweep all of B, so
+// each A block is read from DRAM once and B stays resident in L2; with M
+// fastest the layer's 84 MB activation operand was re-read per column block):
 //   warp 0        TMA producer: A tile 128 x 256 fp4 and B tile 256 x 256 fp4
 //                 (128-byte rows, 128B swizzle) plus the E4M3 scale blocks
 //                 they need (untiled bulk copies of the tensor-core scale
@@ -237,7 +240,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       for (int s = 0; s < STAGES; ++s) issued[s] = false, last_round[s] = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        const int mb = tile % p.num_m, nb = tile / p.num_m;
+        const int mb = tile / p.num_n, nb = tile % p.num_n;
         const int b0 = (nb * BN) / 128;                 // first 128-row scale block of B
         const int nh = min(2, sf_blocks_n - b0);
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
@@ -353,7 +356,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     const int half = ew >> 2;             // columns half*128 .. half*128+127
     uint32_t tile_iter = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
-      const int mb = tile % p.num_m, nb = tile / p.num_m;
+      const int mb = tile / p.num_n, nb = tile % p.num_n;
       const int m = mb * BM + quad * 32 + lane;
       const int nw0 = nb * BN + half * 128;   // first column of this warp
       // resolve the segment before waiting: fast path when all 128 columns

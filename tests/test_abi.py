@@ -75,6 +75,8 @@ def test_bad_arguments_are_rejected_before_launch(L):
     # delta rule: unsupported head dims
     assert L.gdn_delta_rule_fwd(null, null, null, 96, 96, 96, null, null, null, 1, 1, 1, 96, 64, 1,
                                 null, null, null, 0, null) == 2
+    # watchdog self-test: poll limit out of range
+    assert L.gdn_selftest_bounded_wait(0, null) == 1
     # gates: H must be positive
     assert L.gdn_gates(null, null, 4, 0, null, null, null, null, null) == 1
     # layer: workspace missing
