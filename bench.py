@@ -31,6 +31,10 @@ METRIC = "GDN W4A4 layer prefill tokens/s"
 UNIT = "tokens/s"
 WORKLOAD = dict(B=4, T=8192, d_model=5120, H=32, dk=128, dv=128)
 WORKLOAD_NAME = "gdn_w4a4_layer_prefill B=4 T=8192 d_model=5120 H=32 dk=dv=128"
+# kernels of ours one layer forward launches: amax(x), quantize(x), q/k/v/a/b GEMM,
+# scan, quantize(o) with the scan's amax, output GEMM (the two amax words are
+# cleared with cudaMemsetAsync, which launches none of ours)
+LAUNCHES_PER_LAYER_STEP = 6
 CPU_SAMPLE_T = 256            # tokens of one sequence for the oracle sample
 
 
@@ -114,20 +118,28 @@ def stage_costs(B, T, d_model, H, dk, dv):
     }
 
 
-def traffic_from_profiles(kernel):
-    """dram bytes per launch from the committed ncu summary, if the kernel
-    source it was taken from is unchanged."""
+def source_digest(files):
+    """sha256 (first 16 hex digits) of the kernel sources a profile was taken
+    from, concatenated in the given order."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "nvfp4_w4a4_gated_quant_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(stage):
+    """DRAM bytes (read + write) per launch of a layer stage from the committed
+    ncu summary, if the kernel sources it was taken from are unchanged."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
-    import hashlib
     with open(path) as f:
-        rec = json.load(f).get(kernel)
+        rec = json.load(f).get(stage)
     if not rec:
         return None
-    src = os.path.join(ROOT, "nvfp4_w4a4_gated_quant_b200", "csrc", rec["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if h == rec["source_sha"] else None
+    return rec["bytes_per_launch"] if source_digest(rec["sources"]) == rec["source_sha"] else None
 
 
 def run_ours(args, rank, world, local_rank):
@@ -186,7 +198,9 @@ def run_ours(args, rank, world, local_rank):
         ("delta_rule", lambda: _lib.gdn_delta_rule_fwd(
             qv[:, :, :HK].view(B, T, H, dk), qv[:, :, HK:2 * HK].view(B, T, H, dk),
             qv[:, :, 2 * HK:].view(B, T, H, dv), la.view(B, T, H), be.view(B, T, H), o=o, S_T=S_T)),
-        ("quant_o", lambda: _lib.gdn_quantize_nvfp4(o.view(M, HV), codes=o_codes, scales=o_scales, g_out=o_g, ws=qws)),
+        # the layer quantizes o with the amax the scan recorded (no amax pass)
+        ("quant_o", lambda: _lib.gdn_quantize_nvfp4(o.view(M, HV), codes=o_codes, scales=o_scales, g_out=o_g, ws=qws,
+                                                    amax=o_amax)),
         ("gemm_out", lambda: _lib.gemm_bf16(o_codes, o_scales, o_g, lw.out_codes, lw.out_scales, lw.g["out"], M, D, HV,
                                             out=y.view(M, D))),
     ]
@@ -205,8 +219,6 @@ def run_ours(args, rank, world, local_rank):
     # ---- warm-up
     for _ in range(args.warmup):
         layer_step()
-        for _, fn in stages:
-            fn()
     _lib.stream_check()
 
     # ---- timed: the product call on device-resident inputs
@@ -227,7 +239,10 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
 
     # ---- stage breakdown: the same calls one by one, events between them
+    o_amax = o.abs().amax().float().reshape(1)
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    for _, fn in stages:
+        fn()
     torch.cuda.synchronize()
     for i in range(args.steps):
         sev[i][0].record(stream)
@@ -304,7 +319,7 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "tensor", "achieved": round(work / (stage_ms[dom] / 1e3) / 1e12, 1), "peak": fp4_peak,
                 "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
-    roof["traffic"] = traffic_from_profiles(kname)
+    roof["traffic"] = traffic_from_profiles(dom)
     roof["kernel"] = f"{dom} ({kname})"
     roof["peak_source"] = (f"{pk['source']}: " + ("hbm_gbs" if bound == "hbm" else
                                                   "4 x bf16_tflops_sustained (FP4 = 4x bf16 nominal)"))
@@ -319,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "e2e": {"value": round(tokens_per_step / (e2e_ms / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2},
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": LAUNCHES_PER_LAYER_STEP * args.steps,
         "roofline": roof,
         "stages": stage_out,
         "clocks": clk,
