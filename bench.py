@@ -392,19 +392,20 @@ def standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps):
     be = torch.rand((B, T, H), generator=g).to(dev)
     o = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
     S = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
-    for _ in range(args.warmup):
-        _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(reps):
-        _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
     nbytes = 4 * B * T * H * d * 2 + 2 * B * T * H * 4 + B * H * d * d * 4
-    gbs = nbytes / (ms / 1e3) / 1e9
-    out["scan_T32768_H16_d128"] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1),
-                                   "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    # the default kernel (tcgen05 for this shape) and the mma.sync one
+    for key, mma_sync in (("scan_T32768_H16_d128", False), ("scan_T32768_H16_d128_mma_sync", True)):
+        for _ in range(args.warmup):
+            _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S, mma_sync=mma_sync)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S, mma_sync=mma_sync)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[key] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
     return out
 
 

@@ -221,9 +221,13 @@ int gdn_gates(const float* a, const float* b, int64_t M, int H,
  * handled); B*H >= 1.  Values of v and of the state must stay inside the
  * FP16 range (|x| < 65504): the chunk contractions run on FP16 tensor-core
  * operands with FP32 accumulation.
+ * Kernels: dk = 128 with dv a multiple of 64 runs on the 5th-generation
+ * tensor cores (tcgen05.mma, state kept in TMEM); other shapes, or the flag
+ * GDN_DR_MMA_SYNC, run the warp-level mma.sync kernel.  Both compute the same
+ * chunk form; they differ in FP32 summation order only.
  * ws     gdn_delta_rule_workspace_size(...) bytes (may be 0 / NULL).
  * ------------------------------------------------------------------------ */
-enum { GDN_DR_L2NORM_QK = 1, GDN_DR_O_FP32 = 2 };
+enum { GDN_DR_L2NORM_QK = 1, GDN_DR_O_FP32 = 2, GDN_DR_MMA_SYNC = 4 };
 
 size_t gdn_delta_rule_workspace_size(int64_t B, int64_t T, int H, int dk, int dv);
 

@@ -20,7 +20,7 @@ DTYPE_BF16, DTYPE_F32 = 0, 1
 SF_TILED, SF_LINEAR = 0, 1
 EPI_STORE_BF16, EPI_STORE_F32, EPI_LOG_ALPHA, EPI_BETA = 0, 1, 2, 3
 MAX_SEGMENTS = 8
-DR_L2NORM_QK, DR_O_FP32 = 1, 2
+DR_L2NORM_QK, DR_O_FP32, DR_MMA_SYNC = 1, 2, 4
 (WS_X_CODES, WS_X_SCALES, WS_X_G, WS_QKV, WS_LOG_ALPHA, WS_BETA, WS_O, WS_O_CODES,
  WS_O_SCALES, WS_O_G, WS_QUANT, WS_SCAN, WS_COUNT) = range(13)
 
@@ -268,10 +268,11 @@ def _token_stride(t, name):
 
 
 def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=False, o=None, S_T=None,
-                       want_state=True, stream=None):
+                       want_state=True, stream=None, mma_sync=False):
     """q, k [B, T, H, dk], v [B, T, H, dv] bf16 (heads contiguous, token stride
     free); log_alpha, beta FP32 [B, T, H] contiguous; S0 FP32 [B, H, dk, dv].
-    Returns (o [B, T, H, dv] bf16 or FP32, S_T FP32 or None)."""
+    ``mma_sync`` selects the warp-level mma.sync kernel where the tcgen05 one
+    would run.  Returns (o [B, T, H, dv] bf16 or FP32, S_T FP32 or None)."""
     lds = []
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
@@ -293,7 +294,7 @@ def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=Fa
         _need(S0, torch.float32, "S0")
         if not S0.is_contiguous():
             raise ValueError("S0 must be contiguous")
-    flags = (DR_L2NORM_QK if l2norm else 0) | (DR_O_FP32 if o_fp32 else 0)
+    flags = (DR_L2NORM_QK if l2norm else 0) | (DR_O_FP32 if o_fp32 else 0) | (DR_MMA_SYNC if mma_sync else 0)
     L = lib()
     wsz = int(L.gdn_delta_rule_workspace_size(B, T, H, dk, dv))
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev) if wsz else None

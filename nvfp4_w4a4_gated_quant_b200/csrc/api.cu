@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tmap.cuh"
 
 namespace gdn {
 
@@ -47,6 +48,20 @@ int current_device() {
   return d;
 }
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
 
 int record_cuda_error(cudaError_t err) {
   snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(err), cudaGetErrorString(err));
@@ -225,7 +240,7 @@ int gdn_delta_rule_fwd(const void* q, const void* k, const void* v, int64_t ld_q
   (void)ws;
   (void)ws_bytes;
   if (B < 0 || T < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
-  if (flags & ~(GDN_DR_L2NORM_QK | GDN_DR_O_FP32)) return GDN_ERR_INVALID_ARG;
+  if (flags & ~(GDN_DR_L2NORM_QK | GDN_DR_O_FP32 | GDN_DR_MMA_SYNC)) return GDN_ERR_INVALID_ARG;
   if ((dk != 32 && dk != 64 && dk != 128) || (dv != 32 && dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED_SHAPE;
   if (B * (int64_t)H > (1 << 30) || T > (int64_t)1 << 40) return GDN_ERR_UNSUPPORTED_SHAPE;
   if (ld_q < (int64_t)H * dk || ld_k < (int64_t)H * dk || ld_v < (int64_t)H * dv) return GDN_ERR_INVALID_ARG;

@@ -753,6 +753,10 @@ int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
                       cudaStream_t stream) {
   const int64_t chains = B * H;
   if (chains == 0) return GDN_OK;
+  // the tensor-core kernel stores o and S_T in 16-byte vectors
+  if (!(flags & GDN_DR_MMA_SYNC) && delta_rule_tc_supported(dk, dv, T) && aligned(o, 16) && (!S_T || aligned(S_T, 16)))
+    return launch_delta_rule_tc(q, k, v, ld_q, ld_k, ld_v, log_alpha, beta, S0, B, T, H, dk, dv, flags, o, S_T,
+                                o_amax, stream);
   // Split d_v so that the CTAs cover the SMs (one CTA per SM).
   const int sms = num_sms();
   int dvs = dv;

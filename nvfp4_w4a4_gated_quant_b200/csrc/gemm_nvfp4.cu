@@ -15,14 +15,17 @@
 //   warp 0        TMA producer: A tile 128 x 256 fp4 and B tile 256 x 256 fp4
 //                 (128-byte rows, 128B swizzle) plus the E4M3 scale blocks
 //                 they need (untiled bulk copies of the tensor-core scale
-//                 layout) into a 4-stage shared-memory ring.  No multicast.
+//                 layout) into a 4-stage shared-memory ring.  The scale
+//                 copies complete on their own barrier, ahead of the 48 KB of
+//                 operand tiles.  No multicast.
 //   warps 12..15  scale loaders, one per 32-lane TMEM quarter: as soon as a
-//                 stage lands they read its scales from shared memory into
-//                 registers, then, once one of three TMEM scale buffers is
+//                 stage's scales land they read them from shared memory into
+//                 registers, then, once one of five TMEM scale buffers is
 //                 free, write them with tcgen05.st, replicated into the four
-//                 quarters (the layout the block-scaled MMA reads).  Warp
-//                 stores keep these copies off the MMA pipe, where
-//                 tcgen05.cp serialises with the MMAs.
+//                 quarters (the layout the block-scaled MMA reads), while the
+//                 operand tiles are still in flight.  Warp stores keep these
+//                 copies off the MMA pipe, where tcgen05.cp serialises with
+//                 the MMAs.
 //   warp 1        TMEM owner and MMA issuer:
 //                 tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128,
 //                 N=256, K=64) into a 128 x 256 FP32 accumulator in TMEM;
@@ -41,14 +44,13 @@
 // TMEM: accumulator at columns 0..255, scale buffers at 256 + 48b.
 // Every mbarrier wait is bounded; a wait that runs out records
 // GDN_ERR_TIMEOUT, raises a CTA-wide abort flag and every role drains out.
-#include <cuda.h>
-#include <cudaTypedefs.h>
+#include <cstring>
 
-#include <mutex>
 
 #include "common.cuh"
 #include "gate_math.cuh"
 #include "kernels.h"
+#include "tmap.cuh"
 
 namespace gdn {
 namespace {
@@ -57,7 +59,14 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 256;                 // fp4 elements per stage (128 bytes per row)
 constexpr int KSTEP = 64;               // K of one MMA
-constexpr int STAGES = 4;
+#ifndef GDN_GEMM_TMA_STORE
+#define GDN_GEMM_TMA_STORE 1
+#endif
+#ifndef GDN_GEMM_STAGES
+#define GDN_GEMM_STAGES (GDN_GEMM_TMA_STORE ? 3 : 4)
+#endif
+constexpr int STAGES = GDN_GEMM_STAGES;
+constexpr bool TMA_STORE = GDN_GEMM_TMA_STORE != 0;
 constexpr int A_BYTES = BM * BK / 2;    // 16 KiB
 constexpr int B_BYTES = BN * BK / 2;    // 32 KiB
 constexpr int NUM_THREADS = 512;
@@ -74,7 +83,8 @@ constexpr uint32_t SFB_PER_K = BN / 32;
 static_assert(SF_COL + SF_NBUF * SF_BUF <= TMEM_COLS, "TMEM budget");
 
 struct SegSmem {
-  int n_begin, n_end, kind, pad;
+  int n_begin, n_end, kind;
+  int tma;                // bf16 segment with an output tensor map
   float alpha;            // g_a * g_b of the segment
   int64_t ld_out;
   void* out;
@@ -85,12 +95,23 @@ struct SegSmem {
 constexpr int SFA_BYTES = (BK / KSTEP) * 512;      // 2 KiB
 constexpr int SFB_BYTES = 2 * (BK / KSTEP) * 512;  // two 128-row scale blocks, 4 KiB
 
+// Epilogue staging for TMA stores: one 32-row x 64-column bf16 box (4 KiB,
+// 128-byte swizzle) per epilogue warp.
+constexpr int STG_BYTES = 32 * 64 * 2;
+constexpr int STAGING_BYTES = TMA_STORE ? NUM_EPI_WARPS * STG_BYTES : 0;
+
 constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ +
-                              (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 512 +
+                              (size_t)STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + STAGING_BYTES + 512 +
                               GDN_MAX_SEGMENTS * sizeof(SegSmem);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// Output tensor maps of the bf16 segments (TMA-store epilogue).
+struct OutMaps {
+  CUtensorMap m[GDN_MAX_SEGMENTS];
+};
 
 struct Segment {
-  int n_begin, n_end, kind;
+  int n_begin, n_end, kind, tma;
   const float* g_b;
   void* out;
   int64_t ld_out;
@@ -161,24 +182,38 @@ __device__ __forceinline__ void epilogue_store_one(const SegSmem& sg, int m, int
   }
 }
 
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(tmap), "r"(src),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ uint32_t word(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                  const __grid_constant__ Params p) {
+                  const __grid_constant__ Params p, const __grid_constant__ OutMaps om) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSFA = sB + STAGES * B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-  SegSmem* segs = reinterpret_cast<SegSmem*>(sSFB + STAGES * SFB_BYTES);
+  uint8_t* staging = sSFB + STAGES * SFB_BYTES;   // 1024-aligned: every stage size is a multiple of 1 KiB
+  SegSmem* segs = reinterpret_cast<SegSmem*>(staging + STAGING_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(segs + GDN_MAX_SEGMENTS);
   uint64_t* empty = full + STAGES;
-  uint64_t* sf_full = empty + STAGES;      // [3] a scale buffer is filled
-  uint64_t* sf_free = sf_full + SF_NBUF;   // [3] the MMAs that read a buffer are done
+  uint64_t* sf_land = empty + STAGES;      // [STAGES] a stage's scale copies have landed
+  uint64_t* sf_full = sf_land + STAGES;    // [SF_NBUF] a TMEM scale buffer is filled
+  uint64_t* sf_free = sf_full + SF_NBUF;   // [SF_NBUF] the MMAs that read a buffer are done
   uint64_t* acc_full = sf_free + SF_NBUF;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(acc_empty + 1);
@@ -191,6 +226,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_land[s], 1);
     }
     for (int b = 0; b < SF_NBUF; ++b) {
       mbar_init(&sf_full[b], 4);
@@ -207,6 +243,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     d.n_begin = g.n_begin;
     d.n_end = g.n_end;
     d.kind = g.kind;
+    d.tma = g.tma;
     d.alpha = __fmul_rn(*p.g_a, *g.g_b);
     d.ld_out = g.ld_out;
     d.out = g.out;
@@ -217,6 +254,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
   }
+  if (TMA_STORE && warp == EPI_WARP0 && lane < p.n_segs && p.segs[lane].tma) prefetch_tmap(&om.m[lane]);
   if (warp == 1) {
     tmem_alloc(tmem_ptr, TMEM_COLS);
     tmem_relinquish();
@@ -248,14 +286,14 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           const uint32_t round = it / STAGES;
           if (!wait_or_abort(&empty[s], (round & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
           const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
-          const uint32_t bytes = A_BYTES + B_BYTES + (uint32_t)nks * 512u * (1u + (uint32_t)nh);
-          mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], kb * (BK / 2), mb * BM);
-          tma_load_2d(sB + s * B_BYTES, &tmap_b, &full[s], kb * (BK / 2), nb * BN);
-          bulk_load(sSFA + s * SFA_BYTES, p.sfa + ((int64_t)mb * p.kc + kb * 4) * 512, nks * 512, &full[s]);
+          mbar_arrive_expect_tx(&sf_land[s], (uint32_t)nks * 512u * (1u + (uint32_t)nh));
+          bulk_load(sSFA + s * SFA_BYTES, p.sfa + ((int64_t)mb * p.kc + kb * 4) * 512, nks * 512, &sf_land[s]);
           for (int h = 0; h < nh; ++h)
             bulk_load(sSFB + s * SFB_BYTES + h * 2048, p.sfb + ((int64_t)(b0 + h) * p.kc + kb * 4) * 512,
-                      nks * 512, &full[s]);
+                      nks * 512, &sf_land[s]);
+          mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+          tma_load_2d(sA + s * A_BYTES, &tmap_a, &full[s], kb * (BK / 2), mb * BM);
+          tma_load_2d(sB + s * B_BYTES, &tmap_b, &full[s], kb * (BK / 2), nb * BN);
           issued[s] = true;
           last_round[s] = round;
         }
@@ -264,6 +302,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       for (int s = 0; s < STAGES; ++s)
         if (issued[s]) {
           for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&full[s], last_round[s] & 1); ++i) __nanosleep(32);
+          for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sf_land[s], last_round[s] & 1); ++i) __nanosleep(32);
         }
     }
     __syncwarp();
@@ -283,7 +322,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         const int s = it % STAGES;
         const uint32_t buf = it % SF_NBUF;
         bool got = true;
-        if (lane == 0) got = wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag);
+        if (lane == 0) got = wait_or_abort(&sf_land[s], (it / STAGES) & 1, p.status, abort_flag);
         if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) { ok = false; break; }
         const uint4* fa = reinterpret_cast<const uint4*>(sSFA + s * SFA_BYTES) + lane;
         const uint4* fb = reinterpret_cast<const uint4*>(sSFB + s * SFB_BYTES) + lane;
@@ -366,8 +405,11 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       if (nw0 < p.N) {
         s0 = find_segment(segs, n_segs, nw0);
         const SegSmem& sg = segs[s0];
-        fast = sg.kind == GDN_EPI_STORE_BF16 && nw0 + 127 < sg.n_end && nw0 + 127 < p.N && (sg.ld_out % 8) == 0 &&
-               ((reinterpret_cast<uintptr_t>(sg.out) + (int64_t)(nw0 - sg.n_begin) * 2) % 16) == 0;
+        if (TMA_STORE)
+          fast = sg.tma && nw0 + 127 < sg.n_end && nw0 + 127 < p.N;
+        else
+          fast = sg.kind == GDN_EPI_STORE_BF16 && nw0 + 127 < sg.n_end && nw0 + 127 < p.N && (sg.ld_out % 8) == 0 &&
+                 ((reinterpret_cast<uintptr_t>(sg.out) + (int64_t)(nw0 - sg.n_begin) * 2) % 16) == 0;
       }
       bool ok = true;
       if (lane == 0) ok = wait_or_abort(acc_full, tile_iter & 1, p.status, abort_flag);
@@ -375,7 +417,47 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
-      if (fast) {
+      if (TMA_STORE && fast) {
+        // two 64-column halves: both TMEM loads of a half in flight at once,
+        // packed to bf16, staged as a 32 x 64 box and stored by TMA (rows
+        // past M are clipped by the tensor map); the accumulator is released
+        // once the second half is in registers
+        const SegSmem& sg = segs[s0];
+        const float alpha = sg.alpha;
+        const uint32_t stg = smem_u32(staging + ew * STG_BYTES);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tbase + hh * 64, r0);
+          tmem_ld_32x32b_x32(tbase + hh * 64 + 32, r1);
+          tc_wait_ld();
+          if (hh == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          uint32_t pk[32];   // bf16 pairs of the 64 columns
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            pk[e] = f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[2 * e]), alpha)) |
+                    (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[2 * e + 1]), alpha)) << 16);
+            pk[16 + e] = f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[2 * e]), alpha)) |
+                         (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[2 * e + 1]), alpha)) << 16);
+          }
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(stg + lane * 128 + ((c ^ (lane & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                         pk[4 * c + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&om.m[s0], stg, nw0 - sg.n_begin + 64 * hh, mb * BM + quad * 32);
+            bulk_commit();
+          }
+        }
+      } else if (fast) {
         const SegSmem& sg = segs[s0];
         const float alpha = sg.alpha;
         uint32_t pk[64];
@@ -424,6 +506,9 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         }
       }
     }
+    // the staging buffer stays valid until the last store has read it
+    if (TMA_STORE && lane == 0) bulk_wait0();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -432,19 +517,6 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
 }
 
 int make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, uint32_t box_rows) {
@@ -459,6 +531,24 @@ int make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return record_cuda_error(cudaErrorInvalidValue);
   return GDN_OK;
+}
+
+// Tensor map of a bf16 output segment: [M rows, n_end - n_begin columns],
+// row stride ld_out, 32 x 64 boxes with the 128-byte swizzle.  Returns false
+// (the segment then takes the per-element store path) when the segment does
+// not meet TMA's alignment rules.
+bool make_out_map(CUtensorMap* map, const gdn_epilogue_segment_t& sg, int64_t M) {
+  auto encode = tensor_map_encoder();
+  if (!encode || sg.kind != GDN_EPI_STORE_BF16 || sg.n_begin % 8 != 0 || (sg.ld_out * 2) % 16 != 0 ||
+      (reinterpret_cast<uintptr_t>(sg.out) % 16) != 0)
+    return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(sg.n_end - sg.n_begin), (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)(sg.ld_out * 2)};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, sg.out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -488,6 +578,9 @@ int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t*
     p.segs[i].A_log = segs[i].A_log;
     p.segs[i].dt_bias = segs[i].dt_bias;
   }
+  OutMaps om;
+  memset(&om, 0, sizeof(om));
+  for (int i = 0; i < n_segs; ++i) p.segs[i].tma = TMA_STORE && make_out_map(&om.m[i], segs[i], M) ? 1 : 0;
   p.status = device_status_word();
   CUtensorMap ta, tb;
   int st = make_codes_map(&ta, A->codes, M, K, BM);
@@ -498,7 +591,7 @@ int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t*
       cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   if (attr_err != cudaSuccess) return record_cuda_error(attr_err);
   const int grid = (int)std::min<int64_t>(p.num_tiles, num_sms());
-  gemm_nvfp4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ta, tb, p);
+  gemm_nvfp4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ta, tb, p, om);
   return check_launch();
 }
 

@@ -3,8 +3,10 @@
 "Anthology of the SOTA, theory-128", section "The account":
 S_t = alpha_t S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T, o_t = S_t^T q_t over
 L2-normalised q, k.  Tolerance: 2e-3 relative Frobenius on o (FP32 output) and
-on the final state, the bound the task states for 32K tokens.  Both sides get
-the same bf16 q / k / v and the same FP32 gates.
+on the final state, the bound stated for 32K tokens.  Both sides get the same
+bf16 q / k / v and the same FP32 gates.  Shapes with d_k = 128 and d_v a
+multiple of 64 run on the tcgen05 kernel by default; every such case is also
+run on the mma.sync kernel (``mma_sync=True``).
 """
 import numpy as np
 import pytest
@@ -35,9 +37,9 @@ def _case(B, T, H, dk, dv, seed, with_s0=False):
     return q, k, v, la, be, S0
 
 
-def _run(q, k, v, la, be, S0, o_fp32=True):
+def _run(q, k, v, la, be, S0, o_fp32=True, mma_sync=False):
     o, S = _lib.gdn_delta_rule_fwd(bf16_cuda(q), bf16_cuda(k), bf16_cuda(v), f32_cuda(la), f32_cuda(be),
-                                   S0=None if S0 is None else f32_cuda(S0), o_fp32=o_fp32)
+                                   S0=None if S0 is None else f32_cuda(S0), o_fp32=o_fp32, mma_sync=mma_sync)
     _lib.stream_check()
     return to_np(o).astype(np.float64), to_np(S).astype(np.float64)
 
@@ -51,26 +53,32 @@ def _run(q, k, v, la, be, S0, o_fp32=True):
     (2, 96, 40, 128, 128, 5, False),    # 80 chains -> whole 128-column state per CTA
     (1, 160, 2, 32, 32, 6, True),       # the tiny layer's head dims
     (1, 100, 3, 64, 64, 7, False),
+    (3, 300, 50, 128, 128, 8, True),    # 150 chains: more CTAs than SMs
 ])
-def test_delta_rule_matches_oracle(B, T, H, dk, dv, seed, s0):
+@pytest.mark.parametrize("mma_sync", [False, True], ids=["tcgen05", "mma_sync"])
+def test_delta_rule_matches_oracle(B, T, H, dk, dv, seed, s0, mma_sync):
+    if mma_sync and dk != 128:
+        pytest.skip("shape runs on the mma.sync kernel anyway")
     q, k, v, la, be, S0 = _case(B, T, H, dk, dv, seed, s0)
-    o, S = _run(q, k, v, la, be, S0)
+    o, S = _run(q, k, v, la, be, S0, mma_sync=mma_sync)
     o_ref, S_ref = delta_rule_chunked(q, k, v, la, be, S0=S0)
     assert rel_fro(o, o_ref) < TOL, rel_fro(o, o_ref)
     assert rel_fro(S, S_ref) < TOL, rel_fro(S, S_ref)
 
 
-def test_delta_rule_bf16_output():
+@pytest.mark.parametrize("mma_sync", [False, True], ids=["tcgen05", "mma_sync"])
+def test_delta_rule_bf16_output(mma_sync):
     q, k, v, la, be, S0 = _case(1, 190, 4, 128, 128, 9)
-    o, _ = _run(q, k, v, la, be, S0, o_fp32=False)
+    o, _ = _run(q, k, v, la, be, S0, o_fp32=False, mma_sync=mma_sync)
     o_ref, _ = delta_rule_chunked(q, k, v, la, be)
     # bf16 storage adds its own rounding (~1.5e-3 relative RMS) on top
     assert rel_fro(o, o_ref) < 3e-3
 
 
-def test_delta_rule_empty_sequence_returns_initial_state():
+@pytest.mark.parametrize("mma_sync", [False, True], ids=["tcgen05", "mma_sync"])
+def test_delta_rule_empty_sequence_returns_initial_state(mma_sync):
     q, k, v, la, be, S0 = _case(1, 0, 2, 128, 128, 10, True)
-    o, S = _run(q, k, v, la, be, S0)
+    o, S = _run(q, k, v, la, be, S0, mma_sync=mma_sync)
     np.testing.assert_array_equal(S, S0)
 
 
@@ -85,15 +93,31 @@ def test_delta_rule_segments_with_state_carry():
     assert rel_fro(S2, S_all) < 1e-3
 
 
-def test_delta_rule_scan_workload_32k():
+@pytest.mark.parametrize("mma_sync", [False, True], ids=["tcgen05", "mma_sync"])
+def test_delta_rule_scan_workload_32k(mma_sync):
     """The scan workload: B=1, T=32768, H=16, d=128 (gates from a, b as the
     layer computes them); o and S_T within 2e-3 of the FP64 oracle."""
     d = inputs.scan_workload()
     la, be = oracle_gates(d["a"], d["b"], d["A_log"], d["dt_bias"])
     la = la.astype(np.float32)
     be = be.astype(np.float32)
-    o, S = _run(d["q"], d["k"], d["v"], la, be, None)
+    o, S = _run(d["q"], d["k"], d["v"], la, be, None, mma_sync=mma_sync)
     o_ref, S_ref = delta_rule_chunked(d["q"], d["k"], d["v"], la, be)
     e_o, e_s = rel_fro(o, o_ref), rel_fro(S, S_ref)
     print(f"scan 32K: rel_fro o {e_o:.3e}  S_T {e_s:.3e}")
     assert e_o < TOL and e_s < TOL
+
+
+def test_delta_rule_strong_and_no_decay():
+    """Gates at the ends of their range: alpha ~ e^-30 per token (the state
+    forgets within a token) and alpha = 1 with beta = 1 (pure delta rule);
+    every exponent the chunk form takes stays <= 0, so both stay finite."""
+    q, k, v, _, _, S0 = _case(1, 190, 4, 128, 128, 13, True)
+    for la_val, be_val in ((-30.0, 0.5), (0.0, 1.0)):
+        la = np.full(q.shape[:3], la_val, np.float32)
+        be = np.full(q.shape[:3], be_val, np.float32)
+        o_ref, S_ref = delta_rule_chunked(q, k, v, la, be, S0=S0)
+        for mma_sync in (False, True):
+            o, S = _run(q, k, v, la, be, S0, mma_sync=mma_sync)
+            assert np.isfinite(o).all() and np.isfinite(S).all()
+            assert rel_fro(o, o_ref) < TOL and rel_fro(S, S_ref) < TOL, (la_val, mma_sync)

@@ -46,7 +46,10 @@ def test_one_hot_layout():
 
 
 @pytest.mark.parametrize("M,N,K,seed", [(64, 196, 256, 0), (200, 300, 320, 1), (257, 513, 1024, 2),
-                                        (128, 256, 64, 3), (5, 12, 192, 4)])
+                                        (128, 256, 64, 3), (5, 12, 192, 4),
+                                        # row strides of a multiple of 16 bytes: the TMA-store epilogue,
+                                        # with ragged rows clipped by the tensor map
+                                        (300, 384, 512, 6), (1000, 1024, 256, 7), (77, 640, 1280, 8)])
 def test_gemm_matches_oracle(M, N, K, seed):
     rng = np.random.default_rng(seed)
     x = inputs.activations(rng, (M, K))
