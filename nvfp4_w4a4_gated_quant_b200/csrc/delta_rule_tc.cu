@@ -25,9 +25,15 @@
 // the B operand of MMA-1.  The 64 x 64 unit-lower-triangular inverse runs on
 // mma.sync in warps 0-3 (diagonal blocks by right-looking substitution, then
 // the off-diagonal blocks level by level) while warps 4-7 turn the state into
-// S_h and apply the chunk's decay to it.  q, k, v arrive by TMA (3-D tensor
-// maps, so the rows past the end of a sequence read as zeros) into 128-byte
-// swizzled staging, one chunk ahead; o leaves by TMA through shared memory.
+// S_h and apply the chunk's decay to it.
+//
+// Pipeline: the chunk inputs are double-buffered.  Chunk ch+1's q and k land
+// by TMA (3-D tensor maps, so rows past the end of a sequence read as zeros)
+// directly in the [K; Q] rows of the other buffer, and its v in the other
+// beta-V tile; while the tensor cores run chunk ch's MMA-b, MMA-1 and MMA-2/3,
+// the CTA normalises those q and k rows in place, scales v by beta and scans
+// the gates.  The state update of chunk ch is waited for only at the top of
+// chunk ch+1.  o leaves by TMA stores through shared memory.
 //
 // TMEM (512 columns): RA = K K^T | Q K^T, later A U;  RB = [Xw; X] K, later
 // [Q; W] S_h;  R2 = [Xw; X] V;  RS = the state.
@@ -49,31 +55,33 @@ constexpr int DK = 128;
 constexpr int NT = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared-memory map (byte offsets from a 1024-aligned base).
+// Shared-memory map (byte offsets from a 1024-aligned base).  The chunk
+// inputs are double-buffered (buffer ch & 1): chunk ch+1's q, k, v land by TMA
+// and are normalised / beta-scaled in place while chunk ch computes.
 template <int DVS>
 struct Map {
   static constexpr uint32_t T3_ATOM = 192 * 128;             // one 64-column atom of [K; Q; W]
-  static constexpr uint32_t T3 = 0;                          // [K; Q; W]: 192 rows x 128 fp16, K-major
-  static constexpr uint32_t P = T3 + 2 * T3_ATOM;            // [A; Xw; X]: 192 rows x 64 fp16
-  static constexpr uint32_t L = P + 192 * 128;               // L: 64 x 64 fp16
-  static constexpr uint32_t BV = L + 64 * 128;               // beta V, later U: 64 tokens x DVS, N-major
-  static constexpr uint32_t UP = BV + 64 * 2 * DVS;          // U' = diag(e^{G_C-G_s}) U; o staging
-  static constexpr uint32_t SH = UP + 64 * 2 * DVS;          // S_h: 128 (d_k) x DVS, N-major
-  static constexpr uint32_t QS = SH + 128 * 2 * DVS;         // raw bf16 q: 2 atoms of 64 rows x 128 B
-  static constexpr uint32_t KS = QS + 2 * 64 * 128;          // raw bf16 k
-  static constexpr uint32_t VS = KS + 2 * 64 * 128;          // raw bf16 v: DVS / 64 atoms
+  static constexpr uint32_t T3_BYTES = 2 * T3_ATOM;
+  static constexpr uint32_t T3 = 0;                          // 2 x [K; Q; W]: 192 rows x 128 fp16, K-major
+  static constexpr uint32_t P = T3 + 2 * T3_BYTES;           // [A; Xw; X]: 192 rows x 64 fp16 (L in X's place)
+  static constexpr uint32_t VB_BYTES = 64 * 2 * DVS;
+  static constexpr uint32_t VB = P + 192 * 128;              // 2 x (v, beta v, then U): 64 tokens x DVS, N-major
+  static constexpr uint32_t UP = VB + 2 * VB_BYTES;          // U' = diag(e^{G_C-G_s}) U
+  static constexpr uint32_t SH = UP + VB_BYTES;              // S_h: 128 (d_k) x DVS, N-major
+  static constexpr uint32_t OS = SH + 128 * 2 * DVS;         // o staging: 32 x 64 bf16 boxes, 4 KiB each
+  static constexpr uint32_t LD32 = OS + (DVS / 64) * 2 * 4096;   // FP32 diagonal 16 x 16 blocks of L
+  static constexpr uint32_t F = LD32 + 4 * 16 * 16 * 4;      // 2 x per-token factors
+  static constexpr uint32_t F_BYTES = 6 * C * 4 + 16;
+  static constexpr uint32_t G2 = 0, G2M1 = C * 4, BE = 2 * C * 4, D1 = 3 * C * 4, EG = 4 * C * 4, DKF = 5 * C * 4,
+                            GC2 = 6 * C * 4;                 // offsets inside one factor block
+  static constexpr uint32_t MISC = F + 2 * F_BYTES;          // mbarriers, tmem ptr, flags
   static constexpr uint32_t LD_BYTES = 4 * 64 * 128 + 64 * 2 * DVS;   // one chunk's TMA bytes
-  static constexpr uint32_t LAR = VS + 64 * 2 * DVS;         // raw log alpha, beta
-  static constexpr uint32_t BER = LAR + C * 4;
-  static constexpr uint32_t G2 = BER + C * 4;                // G_t log2 e
-  static constexpr uint32_t G2M1 = G2 + C * 4;               // G_{t-1} log2 e
-  static constexpr uint32_t BE = G2M1 + C * 4;               // beta_t
-  static constexpr uint32_t D1 = BE + C * 4;                 // beta_t e^{G_{t-1}}
-  static constexpr uint32_t EG = D1 + C * 4;                 // e^{G_t}
-  static constexpr uint32_t DKF = EG + C * 4;                // e^{G_C - G_t}
-  static constexpr uint32_t MISC = DKF + C * 4;              // mbarriers, tmem ptr, flags, G_C
   static constexpr uint32_t BYTES = MISC + 64;
 };
+static_assert(Map<128>::P % 1024 == 0 && Map<128>::VB % 1024 == 0 && Map<128>::UP % 1024 == 0 &&
+                  Map<128>::SH % 1024 == 0 && Map<128>::OS % 1024 == 0 && Map<64>::OS % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
+static_assert(Map<128>::BYTES + 1024 <= 232448, "shared memory budget");
 
 constexpr uint32_t RA = 0, RB = 128, R2 = 256, RS = 384;
 
@@ -167,9 +175,6 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ float2 unpack_h2(uint32_t w) {
-  return __half22float2(*reinterpret_cast<const __half2*>(&w));
-}
 __device__ __forceinline__ void c_to_a(uint32_t (&a)[4], const float (&c0)[4], const float (&c1)[4]) {
   a[0] = pack_h2(c0[0], c0[1]);
   a[1] = pack_h2(c0[2], c0[3]);
@@ -203,11 +208,6 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* f) {
   }
 }
 
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 struct Args {
   const float* log_alpha;
@@ -225,35 +225,56 @@ struct Maps {
   CUtensorMap q, k, v, o;   // 3-D: (feature, token, batch); o only for bf16 output
 };
 
-// The chunk's q, k, v tiles by TMA (thread 0) and its gates by cp.async
-// (warp 1); rows past the end of the sequence arrive as zeros.
+// The chunk's q (rows 64..127) and k (rows 0..63) straight into buffer p of
+// [K; Q; W] and its v into buffer p of VB, by TMA from one thread; rows past
+// the end of the sequence arrive as zeros.
 template <int DVS>
 __device__ __forceinline__ void issue_chunk_loads(uint32_t sb, const Maps& m, const Args& a, int b, int h,
-                                                  int dv_off, int64_t t0, int tid, int warp, int lane) {
+                                                  int dv_off, int64_t t0, int p) {
   using M = Map<DVS>;
-  if (tid == 0) {
-    const uint32_t bar = sb + M::MISC + 8;
-    mbar_arrive_expect_tx(reinterpret_cast<uint64_t*>(__cvta_shared_to_generic(bar)), M::LD_BYTES);
+  const uint32_t bar = sb + M::MISC + 8;
+  mbar_arrive_expect_tx(reinterpret_cast<uint64_t*>(__cvta_shared_to_generic(bar)), M::LD_BYTES);
+  const uint32_t t3 = sb + M::T3 + (uint32_t)p * M::T3_BYTES;
 #pragma unroll
-    for (int at = 0; at < 2; ++at) {
-      tma_load_3d(sb + M::QS + at * 8192, &m.q, bar, h * DK + 64 * at, (int32_t)t0, b);
-      tma_load_3d(sb + M::KS + at * 8192, &m.k, bar, h * DK + 64 * at, (int32_t)t0, b);
-    }
-#pragma unroll
-    for (int at = 0; at < DVS / 64; ++at)
-      tma_load_3d(sb + M::VS + at * 8192, &m.v, bar, h * a.dv + dv_off + 64 * at, (int32_t)t0, b);
+  for (int at = 0; at < 2; ++at) {
+    tma_load_3d(t3 + at * M::T3_ATOM, &m.k, bar, h * DK + 64 * at, (int32_t)t0, b);
+    tma_load_3d(t3 + at * M::T3_ATOM + 64 * 128, &m.q, bar, h * DK + 64 * at, (int32_t)t0, b);
   }
-  if (warp == 1) {
+  const uint32_t vb = sb + M::VB + (uint32_t)p * M::VB_BYTES;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int t = 2 * lane + e;
-      const bool ok = t0 + t < a.T;
-      const int64_t tok = (int64_t)b * a.T + (ok ? t0 + t : 0);
-      cp_async4(sb + M::LAR + t * 4, a.log_alpha + tok * a.H + h, ok);
-      cp_async4(sb + M::BER + t * 4, a.beta + tok * a.H + h, ok);
-    }
-    cp_async_commit();
+  for (int at = 0; at < DVS / 64; ++at)
+    tma_load_3d(vb + at * 8192, &m.v, bar, h * a.dv + dv_off + 64 * at, (int32_t)t0, b);
+}
+
+// In place: bf16 rows of [K; Q] buffer p -> L2-normalised FP16 (rows r0 ..
+// r0+63; four threads per row, 32 columns each).
+template <int DVS>
+__device__ __forceinline__ void normalize_rows(uint32_t t3, int r0, int tid, int l2norm) {
+  using M = Map<DVS>;
+  constexpr int QC = DK / 4;
+  const int pr = tid >> 2, pq = tid & 3;
+  float v[QC];
+  uint32_t off[QC / 8];
+#pragma unroll
+  for (int i = 0; i < QC / 8; ++i) {
+    const int col = pq * QC + 8 * i;
+    off[i] = t3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(r0 + pr, col & 63);
+    unpack_bf16x8(ld_s128(off[i]), &v[8 * i]);
   }
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < QC; i += 2) {
+    s0 = fmaf(v[i], v[i], s0);
+    s1 = fmaf(v[i + 1], v[i + 1], s1);
+  }
+  float ss = s0 + s1;
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  const float n = l2norm ? rsqrtf(ss + 1e-6f) : 1.0f;
+#pragma unroll
+  for (int i = 0; i < QC; ++i) v[i] *= n;
+#pragma unroll
+  for (int i = 0; i < QC / 8; ++i) st_chunk_h(off[i], &v[8 * i]);
 }
 
 // Thread 0 waits (bounded) for the phase of `bar` with the given parity, then
@@ -267,6 +288,70 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, volatil
   return *abort_flag == 0;
 }
 
+// The raw gates of chunk t0 (warp 7: two tokens per lane; zero past the end
+// of the sequence), fetched well before they are needed.
+__device__ __forceinline__ void fetch_gates(const Args& a, int64_t tok0, int h, int64_t t0, int lane, float (&la)[2],
+                                            float (&bs)[2]) {
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int64_t t = t0 + 2 * lane + e;
+    const bool ok = t < a.T;
+    la[e] = ok ? __ldg(a.log_alpha + (tok0 + t) * a.H + h) : 0.0f;
+    bs[e] = ok ? __ldg(a.beta + (tok0 + t) * a.H + h) : 0.0f;
+  }
+}
+
+// Warp 7: the chunk's gate factors into factor block f from the fetched raw
+// gates (an inclusive scan of log alpha, two tokens per lane).
+template <int DVS>
+__device__ __forceinline__ void scan_gates(float* f, const float (&la)[2], const float (&bs)[2], int lane) {
+  using M = Map<DVS>;
+  const float pair = la[0] + la[1];
+  float x = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const float ex = x - pair;
+  const float G0 = ex + la[0], G1 = x;
+  const float GC = __shfl_sync(0xffffffffu, x, 31);
+  const float Gs[2] = {G0, G1}, Gm[2] = {ex, G0};
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int t = 2 * lane + e;
+    f[M::G2 / 4 + t] = Gs[e] * kLog2e;
+    f[M::G2M1 / 4 + t] = Gm[e] * kLog2e;
+    f[M::D1 / 4 + t] = bs[e] * ex2(Gm[e] * kLog2e);
+    f[M::EG / 4 + t] = ex2(Gs[e] * kLog2e);
+    f[M::DKF / 4 + t] = ex2((GC - Gs[e]) * kLog2e);
+  }
+  if (lane == 31) f[M::GC2 / 4] = GC * kLog2e;
+}
+
+// beta o v in place in VB buffer vb, with beta from factor block f (the rows
+// past the end of the sequence hold zeros and get beta 0).
+template <int DVS>
+__device__ __forceinline__ void scale_v(uint32_t vb, const float* f, int tid) {
+  using M = Map<DVS>;
+  for (int i = tid; i < C * DVS / 8; i += NT) {
+    const uint32_t off = (uint32_t)i * 16;
+    const int r = (i >> 3) & 63;             // token row of this 16-byte chunk
+    const float bt = f[M::BE / 4 + r];
+    float x[8];
+    unpack_bf16x8(ld_s128(vb + off), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] *= bt;
+    st_chunk_h(vb + off, x);
+  }
+}
+
+// Every thread waits (bounded) for a chunk's TMA loads; a wait that runs out
+// raises the abort flag, which the CTA reads after its next barrier.
+__device__ __forceinline__ void wait_loads(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (!mbar_wait(bar, parity, status)) *abort_flag = 1;
+}
+
 template <int DVS, bool O_F32>
 __global__ void __launch_bounds__(NT, 1)
     delta_rule_tc_kernel(const __grid_constant__ Args a, const __grid_constant__ Maps maps) {
@@ -278,17 +363,11 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sb = (sraw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sb - sraw);
-  const float* g2 = reinterpret_cast<const float*>(smem + M::G2);
-  const float* g2m1 = reinterpret_cast<const float*>(smem + M::G2M1);
-  const float* be = reinterpret_cast<const float*>(smem + M::BE);
-  const float* d1 = reinterpret_cast<const float*>(smem + M::D1);
-  const float* eg = reinterpret_cast<const float*>(smem + M::EG);
-  const float* dkf = reinterpret_cast<const float*>(smem + M::DKF);
   uint64_t* bar_mma = reinterpret_cast<uint64_t*>(smem + M::MISC);
   uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + M::MISC + 8);
-  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + M::MISC + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + M::MISC + 20);
-  float* gC2 = reinterpret_cast<float*>(smem + M::MISC + 24);
+  uint64_t* bar_3 = reinterpret_cast<uint64_t*>(smem + M::MISC + 16);   // MMA-3 (state update) done
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + M::MISC + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + M::MISC + 28);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -304,6 +383,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0) {
     mbar_init(bar_mma, 1);
     mbar_init(bar_ld, 1);
+    mbar_init(bar_3, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.q);
@@ -315,8 +395,8 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_alloc(tmem_ptr, 512);
     tmem_relinquish();
   }
-  // [A; Xw; X] starts zero: the strictly upper blocks of Xw and X are never
-  // written afterwards.
+  // [A; Xw; X] starts zero: the strictly upper blocks of Xw are never written
+  // afterwards (those of X are rewritten with zeros every chunk).
   for (int i = tid; i < 192 * 128 / 16; i += NT) st_s128(sb + M::P + i * 16, 0u, 0u, 0u, 0u);
   fence_async_smem();
   tc_fence_before();
@@ -345,130 +425,83 @@ __global__ void __launch_bounds__(NT, 1)
   // half only when the slice has 128 columns)
   const bool o_worker = quarter < 2 && (DVS == 128 || colhalf == 0);
   const int o_col0 = (DVS == 128) ? colhalf * 64 : 0;
-  const uint32_t o_stage = sb + M::UP + (uint32_t)((DVS == 128 ? colhalf * 2 : 0) + quarter) * 4096;
+  const uint32_t o_stage = sb + M::OS + (uint32_t)((DVS == 128 ? colhalf * 2 : 0) + quarter) * 4096;
 
   uint32_t amax_bits = 0;
-  uint32_t mma_phase = 0, ld_phase = 0;
+  uint32_t mma_phase = 0;
   const int64_t nchunks = (T + C - 1) / C;
-  if (nchunks > 0) issue_chunk_loads<DVS>(sb, maps, a, b, h, dv_off, 0, tid, warp, lane);
+
+  // chunk loads issued and waited for (uniform across the CTA); chunk i's
+  // load completes phase i of bar_ld
+  int64_t lds_issued = 0, lds_waited = 0;
+  // chunk 0's inputs, prepared before the loop
+  if (nchunks > 0) {
+    if (tid == 64) issue_chunk_loads<DVS>(sb, maps, a, b, h, dv_off, 0, 0);
+    lds_issued = 1;
+    wait_loads(bar_ld, 0, abort_flag, a.status);
+    lds_waited = 1;
+    normalize_rows<DVS>(sb + M::T3, 0, tid, a.l2norm);
+    normalize_rows<DVS>(sb + M::T3, 64, tid, a.l2norm);
+    float* f0 = reinterpret_cast<float*>(smem + M::F);
+    if (warp == 7) {
+      float la[2], bs[2];
+      fetch_gates(a, tok0, h, 0, lane, la, bs);
+      f0[M::BE / 4 + 2 * lane] = bs[0];
+      f0[M::BE / 4 + 2 * lane + 1] = bs[1];
+      scan_gates<DVS>(f0, la, bs, lane);
+    }
+    __syncthreads();
+    scale_v<DVS>(sb + M::VB, f0, tid);
+    fence_async_smem();
+  }
+  float nla[2] = {0.f, 0.f}, nbs[2] = {0.f, 0.f};   // warp 7: the next chunk's raw gates
   tc_fence_before();
 
 #pragma unroll 1
   for (int64_t ch = 0; ch < nchunks; ++ch) {
     const int64_t t0 = ch * C;
     const int valid = (int)(T - t0 < C ? T - t0 : C);
-    cp_async_wait_all();
-    if (!O_F32 && o_worker && lane == 0) bulk_wait_read0();   // o staging (UP) is rewritten in P4
-    if (!cta_wait(bar_ld, ld_phase & 1, abort_flag, a.status)) break;
-    ++ld_phase;
+    const int p = (int)(ch & 1), pn = p ^ 1;
+    const bool has_next = ch + 1 < nchunks;
+    const uint32_t t3 = sb + M::T3 + (uint32_t)p * M::T3_BYTES;
+    const uint32_t t3n = sb + M::T3 + (uint32_t)pn * M::T3_BYTES;
+    const uint32_t vb = sb + M::VB + (uint32_t)p * M::VB_BYTES;
+    const float* fb = reinterpret_cast<const float*>(smem + M::F + (uint32_t)p * M::F_BYTES);
+    const float* g2 = fb + M::G2 / 4;
+    const float* g2m1 = fb + M::G2M1 / 4;
+    const float* be = fb + M::BE / 4;
+    const float* d1 = fb + M::D1 / 4;
+    const float* eg = fb + M::EG / 4;
+    const float* dkf = fb + M::DKF / 4;
 
-    // ------------------------------------------ P0: norms, gates
-    {
-      constexpr int QC = DK / 4;          // 32 columns per thread, 4 threads per row
-      const int pr = tid >> 2, pq = tid & 3;
-      float qv[QC], kv[QC];
-#pragma unroll
-      for (int i = 0; i < QC / 8; ++i) {
-        const int col = pq * QC + 8 * i;
-        const uint32_t off = (uint32_t)(col >> 6) * 8192 + swz(pr, col & 63);
-        unpack_bf16x8(ld_s128(sb + M::QS + off), &qv[8 * i]);
-        unpack_bf16x8(ld_s128(sb + M::KS + off), &kv[8 * i]);
-      }
-      float qs0 = 0.f, qs1 = 0.f, ks0 = 0.f, ks1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < QC; i += 2) {
-        qs0 = fmaf(qv[i], qv[i], qs0);
-        qs1 = fmaf(qv[i + 1], qv[i + 1], qs1);
-        ks0 = fmaf(kv[i], kv[i], ks0);
-        ks1 = fmaf(kv[i + 1], kv[i + 1], ks1);
-      }
-      float qs = qs0 + qs1, ks = ks0 + ks1;
-      qs += __shfl_xor_sync(0xffffffffu, qs, 1);
-      ks += __shfl_xor_sync(0xffffffffu, ks, 1);
-      qs += __shfl_xor_sync(0xffffffffu, qs, 2);
-      ks += __shfl_xor_sync(0xffffffffu, ks, 2);
-      const float nq = a.l2norm ? rsqrtf(qs + 1e-6f) : 1.0f;
-      const float nk = a.l2norm ? rsqrtf(ks + 1e-6f) : 1.0f;
-#pragma unroll
-      for (int i = 0; i < QC; ++i) {
-        qv[i] *= nq;
-        kv[i] *= nk;
-      }
-      // K rows 0..63 and Q rows 64..127 of [K; Q; W]
-#pragma unroll
-      for (int i = 0; i < QC / 8; ++i) {
-        const int col = pq * QC + 8 * i;
-        const uint32_t atom = (uint32_t)(col >> 6) * M::T3_ATOM;
-        st_chunk_h(sb + M::T3 + atom + swz(pr, col & 63), &kv[8 * i]);
-        st_chunk_h(sb + M::T3 + atom + swz(64 + pr, col & 63), &qv[8 * i]);
-      }
-    }
-    // gates: warp 7, two tokens per lane, one inclusive scan of pair sums
-    if (warp == 7) {
-      const float* lar = reinterpret_cast<const float*>(smem + M::LAR);
-      const float* ber = reinterpret_cast<const float*>(smem + M::BER);
-      float* w_g2 = reinterpret_cast<float*>(smem + M::G2);
-      float* w_g2m1 = reinterpret_cast<float*>(smem + M::G2M1);
-      float* w_be = reinterpret_cast<float*>(smem + M::BE);
-      float* w_d1 = reinterpret_cast<float*>(smem + M::D1);
-      float* w_eg = reinterpret_cast<float*>(smem + M::EG);
-      float* w_dkf = reinterpret_cast<float*>(smem + M::DKF);
-      const float la0 = lar[2 * lane], la1 = lar[2 * lane + 1];
-      const float pair = la0 + la1;
-      float x = pair;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      const float ex = x - pair;
-      const float G0 = ex + la0, G1 = x;
-      const float GC = __shfl_sync(0xffffffffu, x, 31);
-      const float b0 = ber[2 * lane], b1 = ber[2 * lane + 1];
-      const float Gs[2] = {G0, G1}, Gm[2] = {ex, G0}, bs[2] = {b0, b1};
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int t = 2 * lane + e;
-        w_g2[t] = Gs[e] * kLog2e;
-        w_g2m1[t] = Gm[e] * kLog2e;
-        w_be[t] = bs[e];
-        w_d1[t] = bs[e] * ex2(Gm[e] * kLog2e);
-        w_eg[t] = ex2(Gs[e] * kLog2e);
-        w_dkf[t] = ex2((GC - Gs[e]) * kLog2e);
-      }
-      if (lane == 31) *gC2 = GC * kLog2e;
-    }
+    // The previous chunk's state update (MMA-3) has finished: its operands in
+    // buffer pn are free for the next chunk's loads and its state is final.
+    if (tid == 0 && ch > 0 && !mbar_wait(bar_3, (uint32_t)(ch - 1) & 1, a.status)) *abort_flag = 1;
     __syncthreads();
-    // beta o V: the staging and the operand share the N-major swizzled layout
-    for (int i = tid; i < C * DVS / 8; i += NT) {
-      const uint32_t off = (uint32_t)i * 16;
-      const int r = (i >> 3) & 63;           // token row of this 16-byte chunk
-      float f[8];
-      unpack_bf16x8(ld_s128(sb + M::VS + off), f);
-      const float bt = be[r];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] *= bt;
-      st_chunk_h(sb + M::BV + off, f);
+    tc_fence_after();
+    if (*abort_flag) break;
+    if (has_next) {
+      if (tid == 64) issue_chunk_loads<DVS>(sb, maps, a, b, h, dv_off, t0 + C, pn);
+      if (warp == 7) fetch_gates(a, tok0, h, t0 + C, lane, nla, nbs);
+      lds_issued = ch + 2;
     }
-    fence_async_smem();
-    __syncthreads();
+    float* fn = reinterpret_cast<float*>(smem + M::F + (uint32_t)pn * M::F_BYTES);
 
     // ------------------------------------------ MMA-a: [K; Q] K^T -> RA
     if (tid == 0) {
-      tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
 #pragma unroll
       for (int j = 0; j < DK / 16; ++j) {
-        const uint64_t d = sdesc(sb + M::T3 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16);
+        const uint64_t d = sdesc(t3 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16);
         mma_f16(tmem + RA, d, d, id, j > 0 ? 1u : 0u);
       }
       tc_commit(bar_mma);
     }
-    // staging consumed: prefetch the next chunk
-    if (ch + 1 < nchunks) issue_chunk_loads<DVS>(sb, maps, a, b, h, dv_off, t0 + C, tid, warp, lane);
     if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
 
     // ------------------------------------------ P1: L and A from RA
+    const uint32_t Xb = sb + M::P + 128 * 128;    // X, and L before it
+    const uint32_t Xwb = sb + M::P + 64 * 128;
     {
       uint32_t r[32];
       tmem_ld_32x32b_x32(tmem + lane_off + RA + colhalf * 32, r);
@@ -483,8 +516,27 @@ __global__ void __launch_bounds__(NT, 1)
           const int s = s0 + i;
           v[i] = (s < t) ? bt * ex2(fminf(gm - g2[s], 0.0f)) * __uint_as_float(r[i]) : 0.0f;
         }
+        // L (strictly lower; zeros elsewhere) in X's place
 #pragma unroll
-        for (int c = 0; c < 4; ++c) st_chunk_h(sb + M::L + swz(t, s0 + 8 * c), &v[8 * c]);
+        for (int c = 0; c < 4; ++c) st_chunk_h(Xb + swz(t, s0 + 8 * c), &v[8 * c]);
+        // row t of its diagonal block in FP32 for the substitution
+        const int blk = t >> 4;
+        if ((blk >> 1) == colhalf) {
+          // the block's 16 columns are the first or second half of this
+          // thread's 32
+          const uint32_t dst = sb + M::LD32 + (uint32_t)(blk * 256 + (t & 15) * 16) * 4;
+          if (blk & 1) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              st_s128(dst + c * 16, __float_as_uint(v[16 + 4 * c]), __float_as_uint(v[17 + 4 * c]),
+                      __float_as_uint(v[18 + 4 * c]), __float_as_uint(v[19 + 4 * c]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              st_s128(dst + c * 16, __float_as_uint(v[4 * c]), __float_as_uint(v[1 + 4 * c]),
+                      __float_as_uint(v[2 + 4 * c]), __float_as_uint(v[3 + 4 * c]));
+          }
+        }
       } else {
         const int t = (quarter - 2) * 32 + lane;
         const float gt = g2[t];
@@ -503,23 +555,15 @@ __global__ void __launch_bounds__(NT, 1)
 
     // ---------------- P2: X = (I + L)^{-1} and Xw = X diag(d1) (warps 0-3)
     //                  || S -> S_h, S *= e^{G_C} (warps 4-7)
-    const uint32_t Xb = sb + M::P + 128 * 128;
-    const uint32_t Xwb = sb + M::P + 64 * 128;
-    const uint32_t Lb = sb + M::L;
     if (warp < 4) {
+      // P_ik = X_ii L_ik needs L_ik before X_ik overwrites it: warp i reads
+      // only its own block row of L, and only before writing that row
       if (lane < 16) {
         // diagonal block `warp`, column j = lane: right-looking substitution
         // over the block's 16 rows in FP32
         const int base = 16 * warp;
         const int j = lane;
-        uint32_t lw[16][8];            // row t of the block: 16 fp16 as 8 half2
-#pragma unroll
-        for (int t = 1; t < 16; ++t) {
-          const uint4 u0 = ld_s128(Lb + swz(base + t, base));
-          const uint4 u1 = ld_s128(Lb + swz(base + t, base + 8));
-          lw[t][0] = u0.x; lw[t][1] = u0.y; lw[t][2] = u0.z; lw[t][3] = u0.w;
-          lw[t][4] = u1.x; lw[t][5] = u1.y; lw[t][6] = u1.z; lw[t][7] = u1.w;
-        }
+        const uint32_t lb = sb + M::LD32 + (uint32_t)warp * 1024;
         float acc[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) acc[t] = (t == j) ? 1.0f : 0.0f;
@@ -529,11 +573,15 @@ __global__ void __launch_bounds__(NT, 1)
           acc[s2] = xs;
 #pragma unroll
           for (int t = s2 + 1; t < 16; ++t) {
-            const float2 lp = unpack_h2(lw[t][s2 >> 1]);
-            acc[t] = fmaf(-((s2 & 1) ? lp.y : lp.x), xs, acc[t]);
+            float lv;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(lv) : "r"(lb + (uint32_t)(t * 16 + s2) * 4));
+            acc[t] = fmaf(-lv, xs, acc[t]);
           }
         }
         const float dj = d1[base + j];
+        __syncwarp(0x0000ffffu);
+        // P_ik below reads this block row's L, and the diagonal block holds no
+        // L entries the other lanes still need (they come from the FP32 copy)
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
           const __half hx = __float2half_rn(acc[t]);
@@ -545,23 +593,31 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      // off-diagonal blocks, one level (distance) at a time; warp i owns block
-      // row i and keeps P_ik = X_ii L_ik in registers
+      // off-diagonal blocks: warp i owns block row i; P_ik = X_ii L_ik for
+      // every k < i is formed first, then block X_ij (i - j = d) at level d:
+      // X_ij = -sum_{k=j}^{i-1} P_ik X_kj, every X_kj from an earlier level
       uint32_t Pk[3][4];
       const int g = lane >> 2, c4 = lane & 3;
-#pragma unroll 1
+      {
+        uint32_t af[4];
+        frag_a(af, Xb, 16 * warp, 16 * warp, lane);
+#pragma unroll
+        for (int dd = 1; dd <= 3; ++dd) {
+          if (dd <= warp) {
+            float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t bf[4];
+            frag_b_kn(bf, Xb, 16 * warp, 16 * (warp - dd), lane);   // still L_ik
+            mma16816(p0, af, bf[0], bf[1]);
+            mma16816(p1, af, bf[2], bf[3]);
+            c_to_a(Pk[dd - 1], p0, p1);
+          }
+        }
+      }
+      __syncwarp();
+#pragma unroll
       for (int d = 1; d < 4; ++d) {
         if (warp >= d) {
           const int i = warp, jb = warp - d;
-          {
-            float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t af[4], bf[4];
-            frag_a(af, Xb, 16 * i, 16 * i, lane);
-            frag_b_kn(bf, Lb, 16 * i, 16 * (i - d), lane);
-            mma16816(p0, af, bf[0], bf[1]);
-            mma16816(p1, af, bf[2], bf[3]);
-            c_to_a(Pk[d - 1], p0, p1);
-          }
           float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int dd = 1; dd <= 3; ++dd) {
@@ -588,7 +644,7 @@ __global__ void __launch_bounds__(NT, 1)
     } else {
       // S (lanes = d_k rows of this quarter, all DVS columns) -> S_h; S *= e^{G_C}
       const int rr = quarter * 32 + lane;
-      const float eC = ex2(*gC2);
+      const float eC = ex2(fb[M::GC2 / 4]);   // published by the barriers above
 #pragma unroll
       for (int n0 = 0; n0 < DVS; n0 += 32) {
         uint32_t r[32];
@@ -612,6 +668,10 @@ __global__ void __launch_bounds__(NT, 1)
         tmem_st_32x32b_x16(tmem + lane_off + RS + n0 + 16, hi);
       }
       tc_wait_st();
+      if (warp == 7 && has_next) {     // the next chunk's beta, for scale_v after the barrier
+        fn[M::BE / 4 + 2 * lane] = nbs[0];
+        fn[M::BE / 4 + 2 * lane + 1] = nbs[1];
+      }
     }
     fence_async_smem();
     tc_fence_before();
@@ -622,13 +682,22 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       constexpr uint32_t idk = idesc_f16(128, DK, 0, 1);
       constexpr uint32_t idv = idesc_f16(128, DVS, 0, 1);
+      // W first (P3 waits for it alone), then U~ (covered by MMA-1's commit)
 #pragma unroll
-      for (int j = 0; j < C / 16; ++j) {
-        const uint64_t ad = sdesc(sb + M::P + 64 * 128 + j * 32, 16);
-        mma_f16(tmem + RB, ad, sdesc(sb + M::T3 + j * 2048, M::T3_ATOM), idk, j > 0 ? 1u : 0u);
-        mma_f16(tmem + R2, ad, sdesc(sb + M::BV + j * 2048, 64 * 128), idv, j > 0 ? 1u : 0u);
-      }
+      for (int j = 0; j < C / 16; ++j)
+        mma_f16(tmem + RB, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(t3 + j * 2048, M::T3_ATOM), idk,
+                j > 0 ? 1u : 0u);
       tc_commit(bar_mma);
+#pragma unroll
+      for (int j = 0; j < C / 16; ++j)
+        mma_f16(tmem + R2, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), idv,
+                j > 0 ? 1u : 0u);
+    }
+    // while the tensor cores work: the next chunk's q rows, normalised in place
+    if (has_next) {
+      wait_loads(bar_ld, (uint32_t)(ch + 1) & 1, abort_flag, a.status);
+      lds_waited = ch + 2;
+      normalize_rows<DVS>(t3n, 64, tid, a.l2norm);
     }
     if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
 
@@ -646,7 +715,7 @@ __global__ void __launch_bounds__(NT, 1)
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(c < 4 ? r0[8 * c + e] : r1[8 * (c - 4) + e]);
-        st_chunk_h(sb + M::T3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(128 + t, col & 63), f);
+        st_chunk_h(t3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(128 + t, col & 63), f);
       }
     }
     fence_async_smem();
@@ -659,9 +728,14 @@ __global__ void __launch_bounds__(NT, 1)
       constexpr uint32_t id = idesc_f16(128, DVS, 0, 1);
 #pragma unroll
       for (int j = 0; j < DK / 16; ++j)
-        mma_f16(tmem + RB, sdesc(sb + M::T3 + 64 * 128 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16),
+        mma_f16(tmem + RB, sdesc(t3 + 64 * 128 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16),
                 sdesc(sb + M::SH + j * 2048, 128 * 128), id, j > 0 ? 1u : 0u);
       tc_commit(bar_mma);
+    }
+    // the next chunk's k rows and (warp 7) its gate factors
+    if (has_next) {
+      normalize_rows<DVS>(t3n, 0, tid, a.l2norm);
+      if (warp == 7) scan_gates<DVS>(fn, nla, nbs, lane);
     }
     if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
 
@@ -686,7 +760,7 @@ __global__ void __launch_bounds__(NT, 1)
             fd[e] = f[e] * dkt;
           }
           const uint32_t off = (uint32_t)(col >> 6) * (64 * 128) + swz(t, col & 63);
-          st_chunk_h(sb + M::BV + off, f);
+          st_chunk_h(vb + off, f);
           st_chunk_h(sb + M::UP + off, fd);
         }
       }
@@ -700,15 +774,20 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       constexpr uint32_t id2 = idesc_f16(128, DVS, 0, 1);
       constexpr uint32_t id3 = idesc_f16(128, DVS, 1, 1);
+      // A U first (P5 waits for it), then the state update on its own barrier
 #pragma unroll
-      for (int j = 0; j < C / 16; ++j) {
-        const uint64_t ub = sdesc(sb + M::BV + j * 2048, 64 * 128);
-        mma_f16(tmem + RA, sdesc(sb + M::P + j * 32, 16), ub, id2, j > 0 ? 1u : 0u);
-        mma_f16(tmem + RS, sdesc(sb + M::T3 + j * 2048, M::T3_ATOM), sdesc(sb + M::UP + j * 2048, 64 * 128), id3,
-                1u);
-      }
+      for (int j = 0; j < C / 16; ++j)
+        mma_f16(tmem + RA, sdesc(sb + M::P + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), id2, j > 0 ? 1u : 0u);
       tc_commit(bar_mma);
+#pragma unroll
+      for (int j = 0; j < C / 16; ++j)
+        mma_f16(tmem + RS, sdesc(t3 + j * 2048, M::T3_ATOM), sdesc(sb + M::UP + j * 2048, 64 * 128), id3, 1u);
+      tc_commit(bar_3);
     }
+    // the next chunk's beta v
+    if (has_next) scale_v<DVS>(sb + M::VB + (uint32_t)pn * M::VB_BYTES, fn, tid);
+    // the previous chunk's o staging must be read out before P5 rewrites it
+    if (!O_F32 && o_worker && lane == 0) bulk_wait_read0();
     if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
 
     // ------------------------------------------ P5: O = e^{G_t} Q S + A U
@@ -740,27 +819,30 @@ __global__ void __launch_bounds__(NT, 1)
         }
       } else {
         // bf16 row of 64 columns -> swizzled 32 x 64 staging box -> TMA store
+        uint32_t rq1[32], ra1[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + RB + o_col0, rq0);
+        tmem_ld_32x32b_x32(tmem + lane_off + RA + o_col0, ra0);
+        tmem_ld_32x32b_x32(tmem + lane_off + RB + o_col0 + 32, rq1);
+        tmem_ld_32x32b_x32(tmem + lane_off + RA + o_col0 + 32, ra1);
+        tc_wait_ld();
+        float am = 0.0f;
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          const int n0 = o_col0 + c0;
-          tmem_ld_32x32b_x32(tmem + lane_off + RB + n0, rq0);
-          tmem_ld_32x32b_x32(tmem + lane_off + RA + n0, ra0);
-          tc_wait_ld();
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float y0 = fmaf(et, __uint_as_float(rq0[8 * c + 2 * e]), __uint_as_float(ra0[8 * c + 2 * e]));
-              const float y1 =
-                  fmaf(et, __uint_as_float(rq0[8 * c + 2 * e + 1]), __uint_as_float(ra0[8 * c + 2 * e + 1]));
-              const uint32_t b0 = f32_to_bf16_bits(y0), b1 = f32_to_bf16_bits(y1);
-              if (t < valid) amax_bits = max(amax_bits, max(b0 & 0x7FFFu, b1 & 0x7FFFu) << 16);
-              w[e] = b0 | (b1 << 16);
-            }
-            st_s128(o_stage + swz(lane, c0 + 8 * c), w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 4; ++e) {
+            const int i = (8 * c + 2 * e) & 31;
+            const uint32_t* rq = c < 4 ? rq0 : rq1;
+            const uint32_t* ra = c < 4 ? ra0 : ra1;
+            const float y0 = fmaf(et, __uint_as_float(rq[i]), __uint_as_float(ra[i]));
+            const float y1 = fmaf(et, __uint_as_float(rq[i + 1]), __uint_as_float(ra[i + 1]));
+            am = fmaxf(am, fmaxf(fabsf(y0), fabsf(y1)));
+            w[e] = pack_bf16x2(y0, y1);
           }
+          st_s128(o_stage + swz(lane, 8 * c), w[0], w[1], w[2], w[3]);
         }
+        // bf16 rounding is monotone: the largest stored |o| is the rounded max
+        if (t < valid) amax_bits = max(amax_bits, f32_to_bf16_bits(am) << 16);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -769,11 +851,12 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
     }
+    fence_async_smem();       // the next chunk's inputs, written in place above
     tc_fence_before();
   }
 
-  cp_async_wait_all();
   if (!O_F32 && o_worker && lane == 0) bulk_wait0();
+  if (tid == 0 && nchunks > 0 && !mbar_wait(bar_3, (uint32_t)(nchunks - 1) & 1, a.status)) *abort_flag = 1;
   __syncthreads();
   tc_fence_after();
   if (a.o_amax) {
@@ -797,8 +880,8 @@ __global__ void __launch_bounds__(NT, 1)
     }
   }
   // a chunk load still in flight after an abort lands before the CTA exits
-  if (tid == 0 && *abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar_ld, ld_phase & 1); ++i) __nanosleep(32);
+  if (tid == 0 && lds_issued > lds_waited) {
+    for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar_ld, (uint32_t)lds_waited & 1); ++i) __nanosleep(32);
   }
   tc_fence_before();
   __syncthreads();

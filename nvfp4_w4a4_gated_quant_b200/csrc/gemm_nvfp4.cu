@@ -439,10 +439,10 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           uint32_t pk[32];   // bf16 pairs of the 64 columns
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            pk[e] = f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[2 * e]), alpha)) |
-                    (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r0[2 * e + 1]), alpha)) << 16);
-            pk[16 + e] = f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[2 * e]), alpha)) |
-                         (f32_to_bf16_bits(__fmul_rn(__uint_as_float(r1[2 * e + 1]), alpha)) << 16);
+            pk[e] = pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * e]), alpha),
+                                __fmul_rn(__uint_as_float(r0[2 * e + 1]), alpha));
+            pk[16 + e] = pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * e]), alpha),
+                                     __fmul_rn(__uint_as_float(r1[2 * e + 1]), alpha));
           }
           if (lane == 0) bulk_wait_read0();
           __syncwarp();
