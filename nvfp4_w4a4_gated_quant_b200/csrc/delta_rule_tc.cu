@@ -346,6 +346,20 @@ __device__ __forceinline__ void scale_v(uint32_t vb, const float* f, int tid) {
   }
 }
 
+// MMA-a of the chunk in [K; Q; W] buffer t3: [K; Q] K^T into TMEM column d
+// (64 columns: K K^T in lanes 0..63, Q K^T in lanes 64..127); one thread.
+template <int DVS>
+__device__ __forceinline__ void issue_mma_a(uint32_t tmem_d, uint32_t t3, uint64_t* bar) {
+  using M = Map<DVS>;
+  constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
+#pragma unroll
+  for (int j = 0; j < DK / 16; ++j) {
+    const uint64_t d = sdesc(t3 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16);
+    mma_f16(tmem_d, d, d, id, j > 0 ? 1u : 0u);
+  }
+  tc_commit(bar);
+}
+
 // Every thread waits (bounded) for a chunk's TMA loads; a wait that runs out
 // raises the abort flag, which the CTA reads after its next barrier.
 __device__ __forceinline__ void wait_loads(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
@@ -368,6 +382,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint64_t* bar_3 = reinterpret_cast<uint64_t*>(smem + M::MISC + 16);   // MMA-3 (state update) done
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + M::MISC + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + M::MISC + 28);
+  uint64_t* bar_a = reinterpret_cast<uint64_t*>(smem + M::MISC + 32);   // MMA-a (K K^T, Q K^T) done
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -384,6 +399,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(bar_mma, 1);
     mbar_init(bar_ld, 1);
     mbar_init(bar_3, 1);
+    mbar_init(bar_a, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.q);
@@ -450,7 +466,13 @@ __global__ void __launch_bounds__(NT, 1)
       f0[M::BE / 4 + 2 * lane + 1] = bs[1];
       scan_gates<DVS>(f0, la, bs, lane);
     }
+    fence_async_smem();      // the normalised rows, for MMA-a
+    tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      issue_mma_a<DVS>(tmem + R2, sb + M::T3, bar_a);
+    }
     scale_v<DVS>(sb + M::VB, f0, tid);
     fence_async_smem();
   }
@@ -480,6 +502,8 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     if (*abort_flag) break;
+    // MMA-a: chunk 0's was issued in the prologue
+    if (tid == 0 && ch > 0) issue_mma_a<DVS>(tmem + R2, t3, bar_a);
     if (has_next) {
       if (tid == 64) issue_chunk_loads<DVS>(sb, maps, a, b, h, dv_off, t0 + C, pn);
       if (warp == 7) fetch_gates(a, tok0, h, t0 + C, lane, nla, nbs);
@@ -487,24 +511,14 @@ __global__ void __launch_bounds__(NT, 1)
     }
     float* fn = reinterpret_cast<float*>(smem + M::F + (uint32_t)pn * M::F_BYTES);
 
-    // ------------------------------------------ MMA-a: [K; Q] K^T -> RA
-    if (tid == 0) {
-      constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
-#pragma unroll
-      for (int j = 0; j < DK / 16; ++j) {
-        const uint64_t d = sdesc(t3 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16);
-        mma_f16(tmem + RA, d, d, id, j > 0 ? 1u : 0u);
-      }
-      tc_commit(bar_mma);
-    }
-    if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
+    if (!cta_wait(bar_a, (uint32_t)ch & 1, abort_flag, a.status)) break;
 
-    // ------------------------------------------ P1: L and A from RA
+    // ------------------------------------------ P1: L and A from R2 (MMA-a)
     const uint32_t Xb = sb + M::P + 128 * 128;    // X, and L before it
     const uint32_t Xwb = sb + M::P + 64 * 128;
     {
       uint32_t r[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + RA + colhalf * 32, r);
+      tmem_ld_32x32b_x32(tmem + lane_off + R2 + colhalf * 32, r);
       tc_wait_ld();
       const int s0 = colhalf * 32;
       float v[32];
@@ -563,20 +577,27 @@ __global__ void __launch_bounds__(NT, 1)
         // over the block's 16 rows in FP32
         const int base = 16 * warp;
         const int j = lane;
-        const uint32_t lb = sb + M::LD32 + (uint32_t)warp * 1024;
+        const float4* lb4 = reinterpret_cast<const float4*>(smem + M::LD32 + warp * 1024);
+        // left-looking: x_t = [t == j] - sum_{s<t} L_ts x_s, x_t = 0 for t < j;
+        // row t of L read as four 16-byte vectors, four partial sums
         float acc[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) acc[t] = (t == j) ? 1.0f : 0.0f;
+        for (int t = 0; t < 16; ++t) {
+          float l[16];
 #pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) {
-          const float xs = (s2 < j) ? 0.0f : acc[s2];
-          acc[s2] = xs;
-#pragma unroll
-          for (int t = s2 + 1; t < 16; ++t) {
-            float lv;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(lv) : "r"(lb + (uint32_t)(t * 16 + s2) * 4));
-            acc[t] = fmaf(-lv, xs, acc[t]);
+          for (int c = 0; c < (t + 3) / 4; ++c) {
+            const float4 v4 = lb4[t * 4 + c];   // ordinary loads: free to issue early
+            l[4 * c] = v4.x; l[4 * c + 1] = v4.y; l[4 * c + 2] = v4.z; l[4 * c + 3] = v4.w;
           }
+          float p0 = (t == j) ? 1.0f : 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
+#pragma unroll
+          for (int s2 = 0; s2 < t; ++s2) {
+            if ((s2 & 3) == 0) p0 = fmaf(-l[s2], acc[s2], p0);
+            if ((s2 & 3) == 1) p1 = fmaf(-l[s2], acc[s2], p1);
+            if ((s2 & 3) == 2) p2 = fmaf(-l[s2], acc[s2], p2);
+            if ((s2 & 3) == 3) p3 = fmaf(-l[s2], acc[s2], p3);
+          }
+          acc[t] = (t < j) ? 0.0f : (p0 + p1) + (p2 + p3);
         }
         const float dj = d1[base + j];
         __syncwarp(0x0000ffffu);
