@@ -102,6 +102,31 @@ class ClockSampler:
                 "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons), "samples": len(rows)}
 
 
+# ---------------------------------------------------- multi-rank plumbing --
+def replica_seed(rank):
+    """Seed of the batch a rank processes: every rank (GPU) runs its own
+    independent batch of the layer workload, so the job scales weakly."""
+    return 3 + rank
+
+
+def max_over_ranks(v, world, device):
+    """The largest of one float over all ranks (the job's time is its slowest
+    rank's)."""
+    if world == 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(total_ms, steps, tokens_per_rank, world):
+    """(whole-job tokens/s, ms per step) from the max-over-ranks time of
+    `steps` steps in which every rank processed `tokens_per_rank` tokens."""
+    ms_per_step = total_ms / steps
+    return tokens_per_rank * world / (ms_per_step / 1e3), ms_per_step
+
+
 # ---------------------------------------------------------------- our path --
 def stage_costs(B, T, d_model, H, dk, dv):
     """Algorithmic bytes (HBM-bound stages) or FLOPs (contractions) of one
@@ -151,7 +176,7 @@ def run_ours(args, rank, world, local_rank):
     W = WORKLOAD
     B, T, D, H, dk, dv = W["B"], W["T"], W["d_model"], W["H"], W["dk"], W["dv"]
     M, HK, HV = B * T, H * dk, H * dv
-    d = inputs.layer_inputs(B, T, D, H, dk, dv, seed=3 + rank)
+    d = inputs.layer_inputs(B, T, D, H, dk, dv, seed=replica_seed(rank))
     stream = torch.cuda.current_stream()
     lw = _lib.QuantizedLayerWeights(d["W"], d["A_log"], d["dt_bias"], H, dk, dv, device=dev)
     x_host = torch.from_numpy(d["x"]).to(torch.bfloat16).pin_memory()
@@ -209,12 +234,6 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -235,8 +254,8 @@ def run_ours(args, rank, world, local_rank):
     _lib.stream_check()
     total_ms = ev[0].elapsed_time(ev[-1])
     step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = max_over_ranks(total_ms)
-    ms_per_step = total_ms / args.steps
+    total_ms = max_over_ranks(total_ms, world, dev)
+    value, ms_per_step = aggregate(total_ms, args.steps, M, world)
 
     # ---- stage breakdown: the same calls one by one, events between them
     o_amax = o.abs().amax().float().reshape(1)
@@ -286,14 +305,13 @@ def run_ours(args, rank, world, local_rank):
     t1.record(s_out)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(t0.elapsed_time(t1)) / args.steps
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / args.steps
 
     # ---- standalone kernels of the GEMM and scan workloads (context keys)
     kernels = standalone_kernels(args, torch, _lib, inputs, dev, stream) if rank == 0 and not args.skip_kernels else {}
 
     clk = clocks.summary()
     tokens_per_step = M * world
-    value = tokens_per_step / (ms_per_step / 1e3)
     pk = peaks()
     fp4_peak = 4.0 * pk["bf16_tflops_sustained"]           # FP4 dense = 4x bf16 (nominal ratio)
     costs = stage_costs(B, T, D, H, dk, dv)
