@@ -108,13 +108,26 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, i
   return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
+// Warp-collective issue: every lane of the warp executes this with the same
+// (warp-uniform) operands and one elected lane issues the MMA, so the
+// descriptors stay in uniform registers instead of being moved there per
+// instruction from one diverged thread.
+__device__ __forceinline__ void mma_f16_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// tcgen05.commit from one elected lane of a converged warp.
+__device__ __forceinline__ void tc_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -347,7 +360,7 @@ __device__ __forceinline__ void scale_v(uint32_t vb, const float* f, int tid) {
 }
 
 // MMA-a of the chunk in [K; Q; W] buffer t3: [K; Q] K^T into TMEM column d
-// (64 columns: K K^T in lanes 0..63, Q K^T in lanes 64..127); one thread.
+// (64 columns: K K^T in lanes 0..63, Q K^T in lanes 64..127); one warp.
 template <int DVS>
 __device__ __forceinline__ void issue_mma_a(uint32_t tmem_d, uint32_t t3, uint64_t* bar) {
   using M = Map<DVS>;
@@ -355,9 +368,9 @@ __device__ __forceinline__ void issue_mma_a(uint32_t tmem_d, uint32_t t3, uint64
 #pragma unroll
   for (int j = 0; j < DK / 16; ++j) {
     const uint64_t d = sdesc(t3 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16);
-    mma_f16(tmem_d, d, d, id, j > 0 ? 1u : 0u);
+    mma_f16_warp(tmem_d, d, d, id, j > 0 ? 1u : 0u);
   }
-  tc_commit(bar);
+  tc_commit_warp(bar);
 }
 
 // Every thread waits (bounded) for a chunk's TMA loads; a wait that runs out
@@ -469,7 +482,7 @@ __global__ void __launch_bounds__(NT, 1)
     fence_async_smem();      // the normalised rows, for MMA-a
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
       issue_mma_a<DVS>(tmem + R2, sb + M::T3, bar_a);
     }
@@ -503,7 +516,7 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
     if (*abort_flag) break;
     // MMA-a: chunk 0's was issued in the prologue
-    if (tid == 0 && ch > 0) issue_mma_a<DVS>(tmem + R2, t3, bar_a);
+    if (warp == 0 && ch > 0) issue_mma_a<DVS>(tmem + R2, t3, bar_a);
     if (has_next) {
       if (tid == 64) issue_chunk_loads<DVS>(sb, maps, a, b, h, dv_off, t0 + C, pn);
       if (warp == 7) fetch_gates(a, tok0, h, t0 + C, lane, nla, nbs);
@@ -699,19 +712,19 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
 
     // ------------------------------------------ MMA-b: [Xw; X] K -> RB, [Xw; X] V -> R2
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t idk = idesc_f16(128, DK, 0, 1);
       constexpr uint32_t idv = idesc_f16(128, DVS, 0, 1);
       // W first (P3 waits for it alone), then U~ (covered by MMA-1's commit)
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
-        mma_f16(tmem + RB, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(t3 + j * 2048, M::T3_ATOM), idk,
+        mma_f16_warp(tmem + RB, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(t3 + j * 2048, M::T3_ATOM), idk,
                 j > 0 ? 1u : 0u);
-      tc_commit(bar_mma);
+      tc_commit_warp(bar_mma);
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
-        mma_f16(tmem + R2, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), idv,
+        mma_f16_warp(tmem + R2, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), idv,
                 j > 0 ? 1u : 0u);
     }
     // while the tensor cores work: the next chunk's q rows, normalised in place
@@ -744,14 +757,14 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
 
     // ------------------------------------------ MMA-1: [Q; W] S_h -> RB
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, DVS, 0, 1);
 #pragma unroll
       for (int j = 0; j < DK / 16; ++j)
-        mma_f16(tmem + RB, sdesc(t3 + 64 * 128 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16),
+        mma_f16_warp(tmem + RB, sdesc(t3 + 64 * 128 + (j >> 2) * M::T3_ATOM + (j & 3) * 32, 16),
                 sdesc(sb + M::SH + j * 2048, 128 * 128), id, j > 0 ? 1u : 0u);
-      tc_commit(bar_mma);
+      tc_commit_warp(bar_mma);
     }
     // the next chunk's k rows and (warp 7) its gate factors
     if (has_next) {
@@ -791,19 +804,19 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
 
     // ------------------------------------------ MMA-2: [A; *] U -> RA;  MMA-3: S += K^T U'
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t id2 = idesc_f16(128, DVS, 0, 1);
       constexpr uint32_t id3 = idesc_f16(128, DVS, 1, 1);
       // A U first (P5 waits for it), then the state update on its own barrier
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
-        mma_f16(tmem + RA, sdesc(sb + M::P + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), id2, j > 0 ? 1u : 0u);
-      tc_commit(bar_mma);
+        mma_f16_warp(tmem + RA, sdesc(sb + M::P + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), id2, j > 0 ? 1u : 0u);
+      tc_commit_warp(bar_mma);
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
-        mma_f16(tmem + RS, sdesc(t3 + j * 2048, M::T3_ATOM), sdesc(sb + M::UP + j * 2048, 64 * 128), id3, 1u);
-      tc_commit(bar_3);
+        mma_f16_warp(tmem + RS, sdesc(t3 + j * 2048, M::T3_ATOM), sdesc(sb + M::UP + j * 2048, 64 * 128), id3, 1u);
+      tc_commit_warp(bar_3);
     }
     // the next chunk's beta v
     if (has_next) scale_v<DVS>(sb + M::VB + (uint32_t)pn * M::VB_BYTES, fn, tid);
