@@ -4,13 +4,16 @@
 // 'Fragile' Recurrence is Actually Robust" -- NVFP4 scales every 16-element
 // block separately.  Two HBM-bound passes:
 //   amax_kernel   max |x| over the tensor (bf16 bit patterns, one atomicMax
-//                 per CTA on the FP32 bits of the result);
-//   quant_kernel  one thread per 16-element block: two 16-byte loads, the
-//                 block scale, eight packed code bytes and one scale byte.
+//                 per CTA on the FP32 bits of the result), four rows per step;
+//   quant_kernel  one thread per 16-element block and row: two 16-byte loads,
+//                 the block scale, eight packed code bytes and one scale byte;
+//                 two rows per step.
+// CTA widths are chosen so the threads tile a row with the fewest left idle.
 // The FP32 operation order is fixed (see gdn.h); divisions and products use
 // the round-to-nearest intrinsics so no contraction or approximation changes
 // a code.  E4M3 and E2M1 rounding use the hardware cvt.rn.satfinite forms.
 #include <float.h>
+#include <stdint.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -59,10 +62,19 @@ template <typename In, typename E>
 __global__ void amax_kernel(const E* __restrict__ x, int64_t rows, int64_t vpr, int64_t ld,
                             unsigned* __restrict__ amax_bits) {
   uint32_t m = 0;
-  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
-    const E* row = x + r * ld;
-    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < vpr; c += (int64_t)gridDim.x * blockDim.x)
-      m = max(m, In::absmax_bits(ld_vec(row + c * In::kPerVec)));
+  // four rows per step: four independent 16-byte loads in flight per thread
+  const int64_t gy = gridDim.y;
+  for (int64_t r = blockIdx.y; r < rows; r += 4 * gy) {
+    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < vpr; c += (int64_t)gridDim.x * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t rr = r + u * gy;
+        v[u] = rr < rows ? ld_vec(x + rr * ld + c * In::kPerVec) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) m = max(m, In::absmax_bits(v[u]));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -157,25 +169,43 @@ __global__ void quant_kernel(const E* __restrict__ x, int64_t rows, int64_t cols
   const int64_t bpr = cols >> 4;  // 16-element blocks per row
   const int64_t kc = cols >> 6;   // 64-element scale chunks per row (TILED)
   // Two rows per step so that each thread has two blocks' loads in flight.
-  for (int64_t r = blockIdx.y; r < rows; r += 2 * (int64_t)gridDim.y) {
-    const int64_t r2 = r + gridDim.y;
-    const bool two = r2 < rows;
+  constexpr int RU = 2;
+  const int64_t gy = gridDim.y;
+  for (int64_t r = blockIdx.y; r < rows; r += RU * gy) {
     for (int64_t j = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; j < bpr; j += (int64_t)gridDim.x * blockDim.x) {
       constexpr int NV = 16 / In::kPerVec;
-      uint4 va[NV], vb[NV];
+      uint4 v[RU][NV];
 #pragma unroll
-      for (int i = 0; i < NV; ++i) va[i] = ld_vec(x + r * ld + j * 16 + i * In::kPerVec);
-      if (two) {
+      for (int u = 0; u < RU; ++u) {
+        const int64_t rr = r + u * gy;
+        if (rr < rows) {
 #pragma unroll
-        for (int i = 0; i < NV; ++i) vb[i] = ld_vec(x + r2 * ld + j * 16 + i * In::kPerVec);
+          for (int i = 0; i < NV; ++i) v[u][i] = ld_vec(x + rr * ld + j * 16 + i * In::kPerVec);
+        }
       }
-      quant_block<In>(va, g_enc, codes + r * (cols >> 1) + j * 8,
-                      tiled ? scales + scale_offset(r + row_off, j, kc) : scales + r * bpr + j);
-      if (two)
-        quant_block<In>(vb, g_enc, codes + r2 * (cols >> 1) + j * 8,
-                        tiled ? scales + scale_offset(r2 + row_off, j, kc) : scales + r2 * bpr + j);
+#pragma unroll
+      for (int u = 0; u < RU; ++u) {
+        const int64_t rr = r + u * gy;
+        if (rr < rows)
+          quant_block<In>(v[u], g_enc, codes + rr * (cols >> 1) + j * 8,
+                          tiled ? scales + scale_offset(rr + row_off, j, kc) : scales + rr * bpr + j);
+      }
     }
   }
+}
+
+// Threads per CTA for rows of n items: the width among a few warp multiples
+// that leaves the fewest idle threads at the end of a row (the layer's rows
+// have 640 vectors and 320 blocks; 256-wide CTAs would idle 17% and 37%).
+int threads_for_row(int64_t n) {
+  const int cands[] = {256, 192, 160, 128, 96, 64};
+  int best = 256;
+  int64_t best_waste = INT64_MAX;
+  for (int t : cands) {
+    const int64_t waste = cdiv(n, t) * t - n;
+    if (waste < best_waste) best = t, best_waste = waste;
+  }
+  return best;
 }
 
 void grid_for_rows(int64_t rows, int64_t per_row_items, int threads, dim3& grid) {
@@ -191,18 +221,19 @@ template <typename In, typename E>
 int launch_quantize_t(const E* x, int64_t rows, int64_t cols, int64_t ld, int mode, const float* g_enc_in,
                     uint8_t* codes, uint8_t* scales, int tiled, int64_t row_off, float* g_out, unsigned* amax_ws,
                     cudaStream_t stream) {
-  const int threads = 256;
   if (mode == GDN_QUANT_DYNAMIC) {
     cudaError_t e = cudaMemsetAsync(amax_ws, 0, sizeof(unsigned), stream);
     if (e != cudaSuccess) return record_cuda_error(e);
     if (rows > 0) {
+      const int at = threads_for_row(cols / In::kPerVec);
       dim3 grid;
-      grid_for_rows(rows, cols / In::kPerVec, threads, grid);
-      amax_kernel<In, E><<<grid, threads, 0, stream>>>(x, rows, cols / In::kPerVec, ld, amax_ws);
+      grid_for_rows(rows, cols / In::kPerVec, at, grid);
+      amax_kernel<In, E><<<grid, at, 0, stream>>>(x, rows, cols / In::kPerVec, ld, amax_ws);
       int st = check_launch();
       if (st) return st;
     }
   }
+  const int threads = threads_for_row(cols / 16);
   dim3 grid;
   grid_for_rows(rows, cols / 16, threads, grid);
   quant_kernel<In, E><<<grid, threads, 0, stream>>>(x, rows, cols, ld, mode, g_enc_in, amax_ws, codes, scales, tiled,
