@@ -122,14 +122,6 @@ __device__ __forceinline__ void mma_f16_warp(uint32_t d_tmem, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// tcgen05.commit from one elected lane of a converged warp.
-__device__ __forceinline__ void tc_commit_warp(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 2^x on the SFU (ex2.approx, relative error ~2^-22); every argument here is
@@ -396,6 +388,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + M::MISC + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + M::MISC + 28);
   uint64_t* bar_a = reinterpret_cast<uint64_t*>(smem + M::MISC + 32);   // MMA-a (K K^T, Q K^T) done
+  uint64_t* bar_b2 = reinterpret_cast<uint64_t*>(smem + M::MISC + 40);  // MMA-b2 (U~) done
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -413,6 +406,7 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(bar_ld, 1);
     mbar_init(bar_3, 1);
     mbar_init(bar_a, 1);
+    mbar_init(bar_b2, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&maps.q);
@@ -711,21 +705,25 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_before();
     __syncthreads();
 
-    // ------------------------------------------ MMA-b: [Xw; X] K -> RB, [Xw; X] V -> R2
+    // ------------------------------------------ MMA-b: [Xw; X] K -> RB (warp 0), [Xw; X] V -> R2 (warp 1)
+    // Two issuing warps: the halves write different TMEM columns, and each
+    // MMA costs its issuing thread about 80 cycles.
     if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t idk = idesc_f16(128, DK, 0, 1);
-      constexpr uint32_t idv = idesc_f16(128, DVS, 0, 1);
-      // W first (P3 waits for it alone), then U~ (covered by MMA-1's commit)
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
         mma_f16_warp(tmem + RB, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(t3 + j * 2048, M::T3_ATOM), idk,
-                j > 0 ? 1u : 0u);
+                     j > 0 ? 1u : 0u);
       tc_commit_warp(bar_mma);
+    } else if (warp == 1) {
+      tc_fence_after();
+      constexpr uint32_t idv = idesc_f16(128, DVS, 0, 1);
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
         mma_f16_warp(tmem + R2, sdesc(sb + M::P + 64 * 128 + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), idv,
-                j > 0 ? 1u : 0u);
+                     j > 0 ? 1u : 0u);
+      tc_commit_warp(bar_b2);
     }
     // while the tensor cores work: the next chunk's q rows, normalised in place
     if (has_next) {
@@ -771,6 +769,8 @@ __global__ void __launch_bounds__(NT, 1)
       normalize_rows<DVS>(t3n, 0, tid, a.l2norm);
       if (warp == 7) scan_gates<DVS>(fn, nla, nbs, lane);
     }
+    // MMA-1, and U~ (issued by warp 1: MMA-1's commit does not cover it)
+    if (tid == 0 && !mbar_wait(bar_b2, (uint32_t)ch & 1, a.status)) *abort_flag = 1;
     if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
 
     // ------------------------------------------ P4: U = U~ - W S -> U, U'
@@ -803,16 +803,17 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_before();
     __syncthreads();
 
-    // ------------------------------------------ MMA-2: [A; *] U -> RA;  MMA-3: S += K^T U'
+    // ------------------------------------------ MMA-2: [A; *] U -> RA (warp 0);  MMA-3: S += K^T U' (warp 1)
     if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t id2 = idesc_f16(128, DVS, 0, 1);
-      constexpr uint32_t id3 = idesc_f16(128, DVS, 1, 1);
-      // A U first (P5 waits for it), then the state update on its own barrier
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
         mma_f16_warp(tmem + RA, sdesc(sb + M::P + j * 32, 16), sdesc(vb + j * 2048, 64 * 128), id2, j > 0 ? 1u : 0u);
       tc_commit_warp(bar_mma);
+    } else if (warp == 1) {
+      tc_fence_after();
+      constexpr uint32_t id3 = idesc_f16(128, DVS, 1, 1);
 #pragma unroll
       for (int j = 0; j < C / 16; ++j)
         mma_f16_warp(tmem + RS, sdesc(t3 + j * 2048, M::T3_ATOM), sdesc(sb + M::UP + j * 2048, 64 * 128), id3, 1u);

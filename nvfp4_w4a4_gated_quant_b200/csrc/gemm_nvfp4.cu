@@ -357,35 +357,36 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------- MMA issuer
-      uint32_t it = 0, tile_iter = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
-        if (!wait_or_abort(acc_empty, (tile_iter & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t acc = tmem + ACC_COL;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t buf = it % SF_NBUF;
-          if (!wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag) ||
-              !wait_or_abort(&sf_full[buf], (it / SF_NBUF) & 1, p.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
-          const uint32_t a_s = smem_u32(sA + s * A_BYTES);
-          const uint32_t b_s = smem_u32(sB + s * B_BYTES);
-          const uint32_t sf = tmem + SF_COL + buf * SF_BUF;
-          for (int j = 0; j < nks; ++j)
-            tc_mma_nvf4(acc, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc, sf + j * 4,
-                        sf + SFB_OFF + j * SFB_PER_K, (kb > 0 || j > 0) ? 1u : 0u);
-          tc_commit(&empty[s]);
-          tc_commit(&sf_free[buf]);
+    // --------------------------------------------------------- MMA issuer
+    // The whole warp runs this loop (every lane polls the same barriers);
+    // one elected lane issues each MMA and commit.
+    uint32_t it = 0, tile_iter = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tile_iter) {
+      if (!wait_or_abort(acc_empty, (tile_iter & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t acc = tmem + ACC_COL;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t buf = it % SF_NBUF;
+        if (!wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag) ||
+            !wait_or_abort(&sf_full[buf], (it / SF_NBUF) & 1, p.status, abort_flag)) {
+          ok = false;
+          break;
         }
-        if (ok) tc_commit(acc_full);
+        __syncwarp();
+        tc_fence_after();
+        const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
+        const uint32_t a_s = smem_u32(sA + s * A_BYTES);
+        const uint32_t b_s = smem_u32(sB + s * B_BYTES);
+        const uint32_t sf = tmem + SF_COL + buf * SF_BUF;
+        for (int j = 0; j < nks; ++j)
+          tc_mma_nvf4_warp(acc, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc, sf + j * 4,
+                           sf + SFB_OFF + j * SFB_PER_K, (kb > 0 || j > 0) ? 1u : 0u);
+        tc_commit_warp(&empty[s]);
+        tc_commit_warp(&sf_free[buf]);
       }
+      if (ok) tc_commit_warp(acc_full);
     }
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
