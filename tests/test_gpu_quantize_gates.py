@@ -128,6 +128,34 @@ def test_quantize_full_layer_activation_sampled_rows():
     assert to_np(g)[0] == np.float32(np.float32(1) / g_enc)
 
 
+@pytest.mark.parametrize("rows,cols", [(32768, 5120), (4099, 320), (1000, 5120), (7, 64)])
+def test_quantize_dynamic_visits_every_row_once(rows, cols):
+    """The dynamic path (amax pass, then quant pass) and the given-amax path
+    (quant pass only) must, with the same amax, write the same codes and
+    scales into buffers that start out different: no row is skipped or
+    written from another row, at the layer's size and at ragged ones."""
+    if rows == 32768:
+        x = inputs.layer_workload()["x"].reshape(-1, 5120)
+    else:
+        x = inputs.activations(np.random.default_rng(rows), (rows, cols))
+    xd = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    nsf = _lib.scales_tiled_bytes(rows, cols)
+    c_dyn = torch.zeros((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    s_dyn = torch.zeros(nsf, dtype=torch.uint8, device="cuda")
+    c_amx = torch.full((rows, cols // 2), 0xFF, dtype=torch.uint8, device="cuda")
+    s_amx = torch.full((nsf,), 0xFF, dtype=torch.uint8, device="cuda")
+    _, _, g_dyn = _lib.gdn_quantize_nvfp4(xd, codes=c_dyn, scales=s_dyn)
+    amax = xd.float().abs().amax().reshape(1)
+    _, _, g_amx = _lib.gdn_quantize_nvfp4(xd, codes=c_amx, scales=s_amx, amax=amax)
+    torch.cuda.synchronize()
+    assert torch.equal(c_dyn, c_amx)
+    # tiled padding rows past `rows` are never written; compare the real ones
+    lin_dyn = tiled_to_linear(to_np(s_dyn), rows, cols)
+    lin_amx = tiled_to_linear(to_np(s_amx), rows, cols)
+    np.testing.assert_array_equal(lin_dyn, lin_amx)
+    assert to_np(g_dyn)[0].view(np.uint32) == to_np(g_amx)[0].view(np.uint32)
+
+
 # ------------------------------------------------------------------ gates --
 def test_gates_against_oracle():
     rng = np.random.default_rng(11)
