@@ -282,12 +282,12 @@ __device__ __forceinline__ void normalize_rows(uint32_t t3, int r0, int tid, int
   for (int i = 0; i < QC / 8; ++i) st_chunk_h(off[i], &v[8 * i]);
 }
 
-// Thread 0 waits (bounded) for the phase of `bar` with the given parity, then
-// the CTA synchronises; returns false on every thread when the wait ran out.
+// Every thread waits (bounded) for the phase of `bar` with the given parity,
+// then the CTA synchronises; returns false on every thread when the wait ran
+// out.  (Every thread polling measured ~1% faster on the layer shape than
+// thread 0 polling while the others sit in the barrier.)
 __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
-  if (threadIdx.x == 0) {
-    if (!mbar_wait(bar, parity, status)) *abort_flag = 1;
-  }
+  if (!mbar_wait(bar, parity, status)) *abort_flag = 1;
   __syncthreads();
   tc_fence_after();
   return *abort_flag == 0;
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(NT, 1)
 
     // The previous chunk's state update (MMA-3) has finished: its operands in
     // buffer pn are free for the next chunk's loads and its state is final.
-    if (tid == 0 && ch > 0 && !mbar_wait(bar_3, (uint32_t)(ch - 1) & 1, a.status)) *abort_flag = 1;
+    if (ch > 0 && !mbar_wait(bar_3, (uint32_t)(ch - 1) & 1, a.status)) *abort_flag = 1;
     __syncthreads();
     tc_fence_after();
     if (*abort_flag) break;
@@ -770,7 +770,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (warp == 7) scan_gates<DVS>(fn, nla, nbs, lane);
     }
     // MMA-1, and U~ (issued by warp 1: MMA-1's commit does not cover it)
-    if (tid == 0 && !mbar_wait(bar_b2, (uint32_t)ch & 1, a.status)) *abort_flag = 1;
+    if (!mbar_wait(bar_b2, (uint32_t)ch & 1, a.status)) *abort_flag = 1;
     if (!cta_wait(bar_mma, mma_phase++ & 1, abort_flag, a.status)) break;
 
     // ------------------------------------------ P4: U = U~ - W S -> U, U'
