@@ -297,14 +297,15 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         const uint32_t round = it / STAGES;
         if (!wait_or_abort_warp(&empty[s], (round & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
         const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
+        mbar_arrive_expect_tx_warp(&full[s], A_BYTES + B_BYTES);
+        tma_load_2d_warp(sA + s * A_BYTES, &tmap_a, &full[s], kb * (BK / 2), mb * BM);
+        tma_load_2d_warp(sB + s * B_BYTES, &tmap_b, &full[s], kb * (BK / 2), nb * BN);
+        // the stage's scales after its operand tiles (248 -> 246 us)
         mbar_arrive_expect_tx_warp(&sf_land[s], (uint32_t)nks * 512u * (1u + (uint32_t)nh));
         bulk_load_warp(sSFA + s * SFA_BYTES, p.sfa + ((int64_t)mb * p.kc + kb * 4) * 512, nks * 512, &sf_land[s]);
         for (int h = 0; h < nh; ++h)
           bulk_load_warp(sSFB + s * SFB_BYTES + h * 2048, p.sfb + ((int64_t)(b0 + h) * p.kc + kb * 4) * 512,
                          nks * 512, &sf_land[s]);
-        mbar_arrive_expect_tx_warp(&full[s], A_BYTES + B_BYTES);
-        tma_load_2d_warp(sA + s * A_BYTES, &tmap_a, &full[s], kb * (BK / 2), mb * BM);
-        tma_load_2d_warp(sB + s * B_BYTES, &tmap_b, &full[s], kb * (BK / 2), nb * BN);
         issued[s] = true;
         last_round[s] = round;
       }
