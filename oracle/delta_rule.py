@@ -12,7 +12,10 @@ Readings where the pages are silent:
     head) over d_k, eps = 1e-6;
   * no 1/sqrt(d_k) factor on q (the output is S_t^T q_t as written);
   * the correction reads the *undecayed* S_{t-1} (literal form above), not
-    alpha_t S_{t-1};
+    alpha_t S_{t-1}.  The other common reading, where the correction reads
+    the decayed state (S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1}
+    + beta_t k_t v_t^T), is available as ``decayed_read=True`` on the
+    sequential form; the two agree when alpha_t = 1;
   * S is d_k x d_v; S_0 = 0 unless given.
 
 Shapes: q, k [B, T, H, dk]; v [B, T, H, dv]; log_alpha, beta [B, T, H];
@@ -45,8 +48,9 @@ def _prep(q, k, v, log_alpha, beta, S0, normalize):
     return q, k, v, la, be, S0, B, T, H, dk, dv
 
 
-def delta_rule_sequential(q, k, v, log_alpha, beta, S0=None, normalize=True):
-    """The literal per-token recurrence, one token at a time."""
+def delta_rule_sequential(q, k, v, log_alpha, beta, S0=None, normalize=True, decayed_read=False):
+    """The literal per-token recurrence, one token at a time.  With
+    ``decayed_read`` the correction reads alpha_t S_{t-1} instead of S_{t-1}."""
     q, k, v, la, be, S0, B, T, H, dk, dv = _prep(q, k, v, log_alpha, beta, S0, normalize)
     S = S0.reshape(B * H, dk, dv).copy()
     o = np.empty((B, T, H, dv))
@@ -58,7 +62,8 @@ def delta_rule_sequential(q, k, v, log_alpha, beta, S0=None, normalize=True):
     of = np.empty((T, B * H, dv))
     for t in range(T):
         kt = kf[t]
-        r = np.matmul(kt[:, None, :], S)[:, 0, :]                 # S_{t-1}^T k_t
+        S_read = S * af[t][:, None, None] if decayed_read else S
+        r = np.matmul(kt[:, None, :], S_read)[:, 0, :]            # S_{t-1}^T k_t (or of alpha_t S_{t-1})
         S *= af[t][:, None, None]                                 # alpha_t S_{t-1}
         S += (bf[t][:, None] * kt)[:, :, None] * (vf[t] - r)[:, None, :]
         of[t] = np.matmul(qf[t][:, None, :], S)[:, 0, :]          # S_t^T q_t

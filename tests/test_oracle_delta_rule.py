@@ -147,3 +147,54 @@ def test_dv_slice_independent():
     o_s, S_s = delta_rule_sequential(q, k, v[..., 4:8], la, be, S0=S0[..., 4:8])
     np.testing.assert_allclose(o_s, o[..., 4:8], atol=1e-13)
     np.testing.assert_allclose(S_s, S[..., 4:8], atol=1e-13)
+
+
+# ---------------------------------------------------------- decayed read --
+# The other reading of the correction term (it reads alpha_t S_{t-1}):
+# S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T.
+
+def test_decayed_read_single_step_matrix_form():
+    """One step against the matrix form written out with an explicit
+    identity, from a nonzero state, alpha != 1."""
+    rng = np.random.default_rng(21)
+    B, H, dk, dv = 2, 3, 7, 5
+    q, k, v, la, be = _rand(rng, B, 1, H, dk, dv)
+    S0 = rng.standard_normal((B, H, dk, dv))
+    o, S = delta_rule_sequential(q, k, v, la, be, S0=S0, decayed_read=True)
+    qh, kh = l2_normalize(q), l2_normalize(k)
+    for b in range(B):
+        for h in range(H):
+            a, bt, kk = np.exp(la[b, 0, h]), be[b, 0, h], kh[b, 0, h]
+            S_want = a * (np.eye(dk) - bt * np.outer(kk, kk)) @ S0[b, h] + bt * np.outer(kk, v[b, 0, h])
+            np.testing.assert_allclose(S[b, h], S_want, rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(o[b, 0, h], S_want.T @ qh[b, 0, h], rtol=1e-12, atol=1e-14)
+
+
+def test_decayed_read_overwrite_invariant_any_alpha():
+    """With beta = 1 and a unit key the decayed-read update returns v_t for
+    k_t whatever alpha_t is; the undecayed read does so only at alpha = 1."""
+    rng = np.random.default_rng(22)
+    B, T, H, dk, dv = 1, 12, 2, 8, 5
+    q, k, v, la, _ = _rand(rng, B, T, H, dk, dv)
+    k = k / np.linalg.norm(k, axis=-1, keepdims=True)
+    be = np.ones((B, T, H))
+    S = rng.standard_normal((B, H, dk, dv))
+    for t in range(T):
+        _, S = delta_rule_sequential(q[:, t:t + 1], k[:, t:t + 1], v[:, t:t + 1], la[:, t:t + 1],
+                                     be[:, t:t + 1], S0=S, normalize=False, decayed_read=True)
+        for h in range(H):
+            np.testing.assert_allclose(S[0, h].T @ k[0, t, h], v[0, t, h], atol=1e-12)
+    _, S_u = delta_rule_sequential(q[:, :1], k[:, :1], v[:, :1], la[:, :1], be[:, :1],
+                                   S0=rng.standard_normal((B, H, dk, dv)), normalize=False)
+    assert np.abs(S_u[0, 0].T @ k[0, 0, 0] - v[0, 0, 0]).max() > 1e-3
+
+
+def test_decayed_read_equals_undecayed_at_alpha_one():
+    rng = np.random.default_rng(23)
+    q, k, v, _, be = _rand(rng, 2, 19, 3, 6, 4)
+    la = np.zeros(be.shape)
+    S0 = rng.standard_normal((2, 3, 6, 4))
+    o1, S1 = delta_rule_sequential(q, k, v, la, be, S0=S0)
+    o2, S2 = delta_rule_sequential(q, k, v, la, be, S0=S0, decayed_read=True)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(S1, S2)
