@@ -424,6 +424,29 @@ def standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps):
         ms = e0.elapsed_time(e1) / reps
         gbs = nbytes / (ms / 1e3) / 1e9
         out[key] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    # one decode step of 64 sequences x 32 heads x d 128 (state updated in
+    # place; 134 MB of state, read and written once per step)
+    B, T, H = 64, 1, 32
+    q = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((B, T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    la = (-torch.rand((B, T, H), generator=g) * 1.5).to(dev)
+    be = torch.rand((B, T, H), generator=g).to(dev)
+    S = (torch.randn((B, H, d, d), generator=g) * 0.1).to(dev)
+    o = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
+    nbytes = B * H * (2 * d * d * 4 + T * (3 * d * 2 + 8 + d * 2))
+    for _ in range(args.warmup):
+        _lib.gdn_delta_rule_step(q, k, v, la, be, S=S, S_out=S, o=o)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        _lib.gdn_delta_rule_step(q, k, v, la, be, S=S, S_out=S, o=o)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["decode_step_B64_H32_d128"] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1),
+                                       "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
     return out
 
 

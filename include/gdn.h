@@ -239,6 +239,38 @@ int gdn_delta_rule_fwd(const void* q, const void* k, const void* v,
                        void* ws, size_t ws_bytes, gdn_stream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * Step 4, token by token (decode): the recurrence itself, without chunking.
+ *
+ * Passage: as gdn_delta_rule_fwd ("Anthology of the SOTA, theory-128",
+ * section "The account").  Each (batch, head) chain keeps its state in
+ * registers across the T tokens of the call and walks them in order:
+ *   r_t = S_{t-1}^T k_t     (alpha_t S_{t-1}^T k_t with GDN_DR_DECAYED_READ,
+ *                            the reading S_t = alpha_t (I - beta_t k_t k_t^T)
+ *                            S_{t-1} + beta_t k_t v_t^T),
+ *   S_t = alpha_t S_{t-1} + beta_t k_t (v_t - r_t)^T,   o_t = S_t^T q_t.
+ * Meant for decode (T = 1) and short continuations after a chunked prefill;
+ * the state is read and written once per call (2 dk dv 4 bytes per chain).
+ *
+ * q, k, v, ld_*    as gdn_delta_rule_fwd (bf16, element (b, t, h, i) at
+ *                  q[(b*T + t)*ld_q + h*dk + i]); element-aligned only.
+ * log_alpha, beta  FP32 [B, T, H] contiguous.
+ * S_in             FP32 [B, H, dk, dv], or NULL for zeros.
+ * S_out            FP32 [B, H, dk, dv], required; may be S_in (in place).
+ * o                [B, T, H, dv] contiguous; bf16, or FP32 with GDN_DR_O_FP32.
+ * flags            GDN_DR_L2NORM_QK | GDN_DR_O_FP32 | GDN_DR_DECAYED_READ.
+ * Supported: dk and dv in {32, 64, 128}; T >= 0 (T = 0 copies S_in to
+ * S_out); 0 <= B*H <= 2^28.  All FP32 arithmetic; exp via CUDA's expf.
+ * ------------------------------------------------------------------------ */
+enum { GDN_DR_DECAYED_READ = 8 };
+
+int gdn_delta_rule_step(const void* q, const void* k, const void* v,
+                        int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                        const float* log_alpha, const float* beta,
+                        const float* S_in, float* S_out,
+                        int64_t B, int64_t T, int H, int dk, int dv,
+                        int flags, void* o, gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * The layer: steps 1-4 and the output projection, in one call.
  *
  *   xq = quant(x); [q|k|v|a|b] = gemm(xq, W_qkvab) with gates in the epilogue;

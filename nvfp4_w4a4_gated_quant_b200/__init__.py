@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     GdnError,
     QuantizedLayerWeights,
     gdn_delta_rule_fwd,
+    gdn_delta_rule_step,
     gdn_gates,
     gdn_gemm_nvfp4,
     gdn_layer_fwd,

@@ -20,7 +20,7 @@ DTYPE_BF16, DTYPE_F32 = 0, 1
 SF_TILED, SF_LINEAR = 0, 1
 EPI_STORE_BF16, EPI_STORE_F32, EPI_LOG_ALPHA, EPI_BETA = 0, 1, 2, 3
 MAX_SEGMENTS = 8
-DR_L2NORM_QK, DR_O_FP32, DR_MMA_SYNC = 1, 2, 4
+DR_L2NORM_QK, DR_O_FP32, DR_MMA_SYNC, DR_DECAYED_READ = 1, 2, 4, 8
 (WS_X_CODES, WS_X_SCALES, WS_X_G, WS_QKV, WS_LOG_ALPHA, WS_BETA, WS_O, WS_O_CODES,
  WS_O_SCALES, WS_O_G, WS_QUANT, WS_SCAN, WS_COUNT) = range(13)
 
@@ -80,6 +80,9 @@ def lib():
             "gdn_delta_rule_fwd": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_i64,
                                                   c_i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                   c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
+            "gdn_delta_rule_step": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_vp,
+                                                   c_i64, c_i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, c_vp, c_vp]),
             "gdn_layer_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(LayerCfg)]),
             "gdn_layer_workspace_offsets": (ctypes.c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(c_i64)]),
             "gdn_layer_fwd": (ctypes.c_int, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerCfg), c_vp, c_vp,
@@ -97,7 +100,8 @@ def lib():
 
 EXPORTED = ("gdn_status_string", "gdn_last_error", "gdn_version", "gdn_stream_check", "gdn_selftest_bounded_wait",
             "gdn_quantize_workspace_size", "gdn_scales_tiled_bytes", "gdn_quantize_nvfp4", "gdn_gemm_nvfp4",
-            "gdn_gates", "gdn_delta_rule_workspace_size", "gdn_delta_rule_fwd", "gdn_layer_workspace_size",
+            "gdn_gates", "gdn_delta_rule_workspace_size", "gdn_delta_rule_fwd", "gdn_delta_rule_step",
+            "gdn_layer_workspace_size",
             "gdn_layer_workspace_offsets", "gdn_layer_fwd", "gdn_layer_fwd_static_ws")
 LAYER_STATIC_WS_BYTES = 32 << 20
 
@@ -302,6 +306,41 @@ def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=Fa
                                _ptr(beta), _ptr(S0), B, T, H, dk, dv, flags, _ptr(o), _ptr(S_T), _ptr(ws), wsz,
                                _stream(stream)))
     return o, S_T
+
+
+def gdn_delta_rule_step(q, k, v, log_alpha, beta, S=None, l2norm=True, o_fp32=False, decayed_read=False, o=None,
+                        S_out=None, stream=None):
+    """The recurrence token by token (decode, short continuations): q, k
+    [B, T, H, dk], v [B, T, H, dv] bf16 (token stride free); log_alpha, beta
+    FP32 [B, T, H]; S FP32 [B, H, dk, dv] entry state or None for zeros.
+    ``S_out`` defaults to a new tensor; pass ``S_out=S`` to update in place.
+    Returns (o [B, T, H, dv] bf16 or FP32, S_out)."""
+    lds = []
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+        if t.dim() != 4:
+            raise ValueError(f"{n} must be [B, T, H, d]")
+        lds.append(_token_stride(t, n))
+    for t, n in ((log_alpha, "log_alpha"), (beta, "beta")):
+        _need(t, torch.float32, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32 if o_fp32 else torch.bfloat16, device=dev)
+    if S_out is None:
+        S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    for t, n in ((S, "S"), (S_out, "S_out")):
+        if t is not None:
+            _need(t, torch.float32, n)
+            if not t.is_contiguous():
+                raise ValueError(f"{n} must be contiguous")
+    flags = (DR_L2NORM_QK if l2norm else 0) | (DR_O_FP32 if o_fp32 else 0) | (DR_DECAYED_READ if decayed_read else 0)
+    check(lib().gdn_delta_rule_step(_ptr(q), _ptr(k), _ptr(v), lds[0], lds[1], lds[2], _ptr(log_alpha), _ptr(beta),
+                                    _ptr(S), _ptr(S_out), B, T, H, dk, dv, flags, _ptr(o), _stream(stream)))
+    return o, S_out
 
 
 # ------------------------------------------------------------------ layer --

@@ -257,4 +257,26 @@ int gdn_delta_rule_fwd(const void* q, const void* k, const void* v, int64_t ld_q
                            flags, o, S_T, nullptr, as_stream(stream));
 }
 
+int gdn_delta_rule_step(const void* q, const void* k, const void* v, int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                        const float* log_alpha, const float* beta, const float* S_in, float* S_out, int64_t B,
+                        int64_t T, int H, int dk, int dv, int flags, void* o, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+  if (flags & ~(GDN_DR_L2NORM_QK | GDN_DR_O_FP32 | GDN_DR_DECAYED_READ)) return GDN_ERR_INVALID_ARG;
+  if ((dk != 32 && dk != 64 && dk != 128) || (dv != 32 && dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (B * (int64_t)H > (1 << 28) || T > (int64_t)1 << 40) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (ld_q < (int64_t)H * dk || ld_k < (int64_t)H * dk || ld_v < (int64_t)H * dv) return GDN_ERR_INVALID_ARG;
+  if (B == 0) return GDN_OK;
+  if (!S_out) return GDN_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!q || !k || !v || !log_alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 2) || !aligned(k, 2) || !aligned(v, 2)) return GDN_ERR_ALIGNMENT;
+    if (!aligned(o, (flags & GDN_DR_O_FP32) ? 4 : 2) || !aligned(log_alpha, 4) || !aligned(beta, 4))
+      return GDN_ERR_ALIGNMENT;
+  }
+  if ((S_in && !aligned(S_in, 4)) || !aligned(S_out, 4)) return GDN_ERR_ALIGNMENT;
+  return launch_delta_rule_step(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                static_cast<const uint16_t*>(v), ld_q, ld_k, ld_v, log_alpha, beta, S_in, S_out, B,
+                                T, H, dk, dv, flags, o, as_stream(stream));
+}
+
 }  // extern "C"

@@ -24,6 +24,12 @@ int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
                       int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
                       cudaStream_t stream);
 
+// The token-by-token recurrence (state in registers; decode and short
+// continuations).
+int launch_delta_rule_step(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
+                           int64_t ld_v, const float* log_alpha, const float* beta, const float* S_in, float* S_out,
+                           int64_t B, int64_t T, int H, int dk, int dv, int flags, void* o, cudaStream_t stream);
+
 // The tcgen05 scan (d_k = 128, d_v % 64 == 0, T < 2^31: its tensor maps take
 // 32-bit token coordinates); launch_delta_rule dispatches to it unless
 // GDN_DR_MMA_SYNC is set.

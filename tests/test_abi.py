@@ -75,6 +75,13 @@ def test_bad_arguments_are_rejected_before_launch(L):
     # delta rule: unsupported head dims
     assert L.gdn_delta_rule_fwd(null, null, null, 96, 96, 96, null, null, null, 1, 1, 1, 96, 64, 1,
                                 null, null, null, 0, null) == 2
+    # delta rule step: unknown flag, unsupported head dim, missing output state
+    assert L.gdn_delta_rule_step(null, null, null, 128, 128, 128, null, null, null, ctypes.c_void_p(256), 1, 1, 1,
+                                 128, 128, 16, null, null) == 1
+    assert L.gdn_delta_rule_step(null, null, null, 96, 96, 96, null, null, null, ctypes.c_void_p(256), 1, 1, 1,
+                                 96, 64, 1, null, null) == 2
+    assert L.gdn_delta_rule_step(null, null, null, 128, 128, 128, null, null, null, null, 1, 0, 1,
+                                 128, 128, 1, null, null) == 1
     # watchdog self-test: poll limit out of range
     assert L.gdn_selftest_bounded_wait(0, null) == 1
     # gates: H must be positive
