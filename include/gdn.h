@@ -275,7 +275,8 @@ int gdn_delta_rule_step(const void* q, const void* k, const void* v,
  *
  *   xq = quant(x); [q|k|v|a|b] = gemm(xq, W_qkvab) with gates in the epilogue;
  *   o  = delta_rule(q, k, v, log_alpha, beta; L2-normalised q, k);
- *   y  = gemm(quant(o), W_out)  (bf16 out).
+ *   y  = gemm(quant(o), W_out)  (bf16 out); quant(o) uses o's own amax, or
+ *        the static encode scale w->o_g_enc when one is given.
  * No short convolution, output gate, norm or residual.
  *
  * Weights are pre-quantized by the caller (gdn_quantize_nvfp4, one call per
@@ -306,6 +307,12 @@ typedef struct {
   const float* g_out;
   const float* A_log;    /* [H] */
   const float* dt_bias;  /* [H] */
+  const float* o_g_enc;  /* NULL: o is quantized with its own amax (dynamic).
+                            Else a device FP32 encode scale for o (a static,
+                            calibrated activation scale): the scan writes o's
+                            NVFP4 codes and scales itself (in its epilogue when
+                            the tensor-core scan runs) and no quantizer pass
+                            runs; the decode scale is 1 / o_g_enc. */
 } gdn_layer_weights_t;
 
 enum {

@@ -48,7 +48,8 @@ class LayerCfg(ctypes.Structure):
 
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_qkvab", Nvfp4), ("g_q", c_vp), ("g_k", c_vp), ("g_v", c_vp), ("g_a", c_vp),
-                ("g_b", c_vp), ("w_out", Nvfp4), ("g_out", c_vp), ("A_log", c_vp), ("dt_bias", c_vp)]
+                ("g_b", c_vp), ("w_out", Nvfp4), ("g_out", c_vp), ("A_log", c_vp), ("dt_bias", c_vp),
+                ("o_g_enc", c_vp)]
 
 
 _LIB = None
@@ -347,7 +348,9 @@ def gdn_delta_rule_step(q, k, v, log_alpha, beta, S=None, l2norm=True, o_fp32=Fa
 class QuantizedLayerWeights:
     """NVFP4 weights of one layer, quantized on the device by the library:
     q, k, v, a, b share one [2*H*dk + H*dv + 2*H, d_model] operand (each with
-    its own decode scale), out is [d_model, H*dv]."""
+    its own decode scale), out is [d_model, H*dv].  ``o_g_enc`` (a 1-element
+    FP32 CUDA tensor, default None) is a static encode scale for the output
+    projection's activation; None quantizes o with its own amax."""
 
     def __init__(self, W, A_log, dt_bias, H, dk, dv, device="cuda", stream=None):
         d_model = W["q"].shape[1]
@@ -368,6 +371,7 @@ class QuantizedLayerWeights:
         self.out_codes, self.out_scales, self.g["out"] = gdn_quantize_nvfp4(wo, stream=stream)
         self.A_log = torch.as_tensor(A_log, dtype=torch.float32).to(device).contiguous()
         self.dt_bias = torch.as_tensor(dt_bias, dtype=torch.float32).to(device).contiguous()
+        self.o_g_enc = None
 
     def struct(self):
         s = LayerWeights()
@@ -377,6 +381,9 @@ class QuantizedLayerWeights:
         s.w_out = Nvfp4(self.out_codes.data_ptr(), self.out_scales.data_ptr())
         s.g_out = self.g["out"].data_ptr()
         s.A_log, s.dt_bias = self.A_log.data_ptr(), self.dt_bias.data_ptr()
+        if self.o_g_enc is not None:
+            _need(self.o_g_enc, torch.float32, "o_g_enc")
+            s.o_g_enc = self.o_g_enc.data_ptr()
         return s
 
 

@@ -44,6 +44,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "quant_math.cuh"
 #include "kernels.h"
 #include "tmap.cuh"
 
@@ -225,6 +226,11 @@ struct Args {
   float* S_T;
   unsigned* o_amax;
   int* status;
+  // fused NVFP4 quantization of the bf16 o (codes == nullptr: off)
+  uint8_t* oq_codes;
+  uint8_t* oq_scales;
+  const float* oq_g_enc;
+  float* oq_g_out;
 };
 struct Maps {
   CUtensorMap q, k, v, o;   // 3-D: (feature, token, batch); o only for bf16 output
@@ -452,6 +458,8 @@ __global__ void __launch_bounds__(NT, 1)
 
   uint32_t amax_bits = 0;
   uint32_t mma_phase = 0;
+  const float oq_genc = a.oq_codes ? *a.oq_g_enc : 1.0f;
+  if (a.oq_codes && blockIdx.x == 0 && tid == 0) *a.oq_g_out = __fdiv_rn(1.0f, oq_genc);
   const int64_t nchunks = (T + C - 1) / C;
 
   // chunk loads issued and waited for (uniform across the CTA); chunk i's
@@ -884,6 +892,21 @@ __global__ void __launch_bounds__(NT, 1)
           tma_store_3d(&maps.o, o_stage, h * a.dv + dv_off + o_col0, (int32_t)(t0 + quarter * 32), b);
           bulk_commit();
         }
+        if (a.oq_codes && t < valid) {
+          // this row's 64 staged bf16 values -> four NVFP4 blocks (codes and
+          // tiled scales of the output projection's activation, K = H*dv)
+          const int64_t row = tok0 + t0 + t;
+          const int64_t HV = (int64_t)a.H * a.dv;
+          const int64_t kcol = (int64_t)h * a.dv + dv_off + o_col0;
+          uint8_t* cp = a.oq_codes + row * (HV >> 1) + (kcol >> 1);
+          uint8_t* sp = a.oq_scales + (row >> 7) * (HV >> 6) * 512 + (kcol >> 6) * 512 + (row & 31) * 16 +
+                        ((row & 127) >> 5) * 4;
+#pragma unroll
+          for (int qb = 0; qb < 4; ++qb) {
+            const uint4 blk[2] = {ld_s128(o_stage + swz(lane, 16 * qb)), ld_s128(o_stage + swz(lane, 16 * qb + 8))};
+            quant_block<Bf16In>(blk, oq_genc, cp + 8 * qb, sp + qb);
+          }
+        }
       }
     }
     fence_async_smem();       // the next chunk's inputs, written in place above
@@ -959,10 +982,11 @@ bool delta_rule_tc_supported(int dk, int dv, int64_t T) { return dk == DK && dv 
 int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                          int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
                          int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const OQuant* oq) {
   const int64_t chains = B * H;
   if (chains == 0) return GDN_OK;
   if (!delta_rule_tc_supported(dk, dv, T)) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (oq && (flags & GDN_DR_O_FP32)) return GDN_ERR_UNSUPPORTED_SHAPE;
   // d_v slices of 128 columns unless the chains leave more than half the SMs idle
   const int sms = num_sms();
   int dvs = (dv % 128 == 0) ? 128 : 64;
@@ -988,6 +1012,12 @@ int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v
   a.S_T = S_T;
   a.o_amax = o_amax;
   a.status = device_status_word();
+  if (oq) {
+    a.oq_codes = oq->codes;
+    a.oq_scales = oq->scales;
+    a.oq_g_enc = oq->g_enc;
+    a.oq_g_out = oq->g_out;
+  }
   if (dvs == 128) return f32 ? launch_dvs<128, true>(a, m, chains, stream) : launch_dvs<128, false>(a, m, chains, stream);
   return f32 ? launch_dvs<64, true>(a, m, chains, stream) : launch_dvs<64, false>(a, m, chains, stream);
 }

@@ -19,10 +19,21 @@ int launch_gates(const float* a, const float* b, int64_t M, int H, const float* 
 int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B, int64_t M, int64_t N,
                       int64_t K, const gdn_epilogue_segment_t* segs, int n_segs, cudaStream_t stream);
 
+// NVFP4 quantization of the scan's bf16 o with a given encode scale: codes
+// [B*T, H*dv/2], TILED scales (K = H*dv), decode scale 1 / g_enc.
+struct OQuant {
+  uint8_t* codes;
+  uint8_t* scales;
+  const float* g_enc;   // device scalar
+  float* g_out;         // device scalar, written: 1 / g_enc
+};
+
+// oq: when given, o (bf16) is also quantized -- inside the tensor-core scan's
+// epilogue, or by a separate given-scale pass when another kernel runs.
 int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                       int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
                       int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
-                      cudaStream_t stream);
+                      cudaStream_t stream, const OQuant* oq = nullptr);
 
 // The token-by-token recurrence (state in registers; decode and short
 // continuations).
@@ -37,6 +48,6 @@ bool delta_rule_tc_supported(int dk, int dv, int64_t T);
 int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                          int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
                          int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
-                         cudaStream_t stream);
+                         cudaStream_t stream, const OQuant* oq = nullptr);
 
 }  // namespace gdn

@@ -111,18 +111,24 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
   st = gdn_gemm_nvfp4(&xa, x_g, &w->w_qkvab, M, NQKV + 2 * H, D, seg, 5, s);
   if (st) return st;
 
-  // The scan records max |o| of the bf16 values it stores, so o is
-  // quantized in one pass (given-amax mode) instead of amax pass + pass.
+  // Dynamic o scale: the scan records max |o| of the bf16 values it stores,
+  // so o is quantized in one pass (given-amax mode) instead of amax pass +
+  // pass.  Static o scale (w->o_g_enc): the scan writes o's codes and scales
+  // itself, and no quantizer pass runs.
   unsigned* o_amax = static_cast<unsigned*>(qws);
   cudaError_t ce = cudaMemsetAsync(o_amax, 0, sizeof(unsigned), reinterpret_cast<cudaStream_t>(s));
   if (ce != cudaSuccess) return record_cuda_error(ce);
+  OQuant oq{o_codes, o_scales, w->o_g_enc, o_g};
   st = launch_delta_rule(qkv, qkv + HK, qkv + 2 * HK, NQKV, NQKV, NQKV, log_alpha, beta, S0, cfg->B, cfg->T, H, dk, dv,
-                         GDN_DR_L2NORM_QK, o, S_T, o_amax, reinterpret_cast<cudaStream_t>(s));
+                         GDN_DR_L2NORM_QK, o, S_T, o_amax, reinterpret_cast<cudaStream_t>(s),
+                         w->o_g_enc ? &oq : nullptr);
   if (st) return st;
 
-  st = gdn_quantize_nvfp4(o, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_GIVEN_AMAX, reinterpret_cast<const float*>(o_amax),
-                          o_codes, o_scales, GDN_SF_TILED, 0, o_g, nullptr, 0, s);
-  if (st) return st;
+  if (!w->o_g_enc) {
+    st = gdn_quantize_nvfp4(o, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_GIVEN_AMAX, reinterpret_cast<const float*>(o_amax),
+                            o_codes, o_scales, GDN_SF_TILED, 0, o_g, nullptr, 0, s);
+    if (st) return st;
+  }
 
   gdn_nvfp4_t oa{o_codes, o_scales};
   gdn_epilogue_segment_t yseg = {0, D, GDN_EPI_STORE_BF16, w->g_out, y, D, nullptr, nullptr};

@@ -146,3 +146,48 @@ def test_layer_workload_sampled():
     np.testing.assert_array_equal(to_np(v["o_codes"][rows_t]), oq["codes"])
     y_gpu = to_np(y.view(M, D)[rows_t])
     assert rel_fro(y_gpu, gemm_bf16(oq, Wq["out"])) < 1e-3
+
+
+@pytest.mark.parametrize("dims", [
+    (2, 200, 512, 4, 128, 128),    # tensor-core scan, 64-column d_v slices, ragged last chunk
+    (2, 70, 512, 40, 128, 128),    # tensor-core scan, whole 128-column slices
+    (1, 96, 256, 2, 32, 32),       # mma.sync scan: o quantized by a given-scale pass
+], ids=["tc_dvs64", "tc_dvs128", "mma_sync"])
+def test_layer_static_o_scale(dims):
+    """A static encode scale for o (gdn_layer_weights_t.o_g_enc): the scan
+    writes o's NVFP4 codes and scales itself.  Given the dynamic run's own
+    scale, every byte and y are identical to the dynamic run; given another
+    scale, the codes and scales equal the oracle's quantization of the same
+    bf16 o with that scale, bit for bit."""
+    B, T, D, H, dk, dv = dims
+    M, HV = B * T, H * dv
+    d = inputs.layer_inputs(B, T, D, H, dk, dv, seed=11)
+    lw = _lib.QuantizedLayerWeights(d["W"], d["A_log"], d["dt_bias"], H, dk, dv)
+    x = torch.from_numpy(d["x"]).cuda().to(torch.bfloat16)
+    y0, S0, ws0 = _lib.gdn_layer_fwd(lw, x)
+    _lib.stream_check()
+    v0 = _ws_views(ws0, dims)
+    o = to_np(v0["o"]).astype(np.float32)
+    g_enc = nvfp4.global_encode_scale(nvfp4.tensor_amax(o))
+    lw.o_g_enc = torch.tensor([g_enc], dtype=torch.float32, device="cuda")
+    y1, S1, ws1 = _lib.gdn_layer_fwd(lw, x)
+    _lib.stream_check()
+    v1 = _ws_views(ws1, dims)
+    assert torch.equal(v1["o"], v0["o"])
+    assert torch.equal(v1["o_codes"], v0["o_codes"])
+    np.testing.assert_array_equal(tiled_to_linear(to_np(v1["o_scales"]), M, HV),
+                                  tiled_to_linear(to_np(v0["o_scales"]), M, HV))
+    assert to_np(v1["o_g"])[0] == to_np(v0["o_g"])[0]
+    assert torch.equal(y1, y0)
+    assert torch.equal(S1, S0)
+    # another static scale: compare with the oracle on the same o
+    g2 = np.float32(g_enc * np.float32(0.37))
+    lw.o_g_enc = torch.tensor([g2], dtype=torch.float32, device="cuda")
+    _, _, ws2 = _lib.gdn_layer_fwd(lw, x)
+    _lib.stream_check()
+    v2 = _ws_views(ws2, dims)
+    o2 = to_np(v2["o"]).astype(np.float32)
+    ref = nvfp4.quantize(o2, g_enc=g2)
+    np.testing.assert_array_equal(to_np(v2["o_codes"]), ref["codes"])
+    np.testing.assert_array_equal(tiled_to_linear(to_np(v2["o_scales"]), M, HV), ref["scales"])
+    assert to_np(v2["o_g"])[0] == np.float32(ref["g"])
