@@ -90,3 +90,33 @@ def test_bad_arguments_are_rejected_before_launch(L):
     cfg = _lib.layer_cfg(1, 64, 256, 2, 128, 128)
     w = _lib.LayerWeights()
     assert L.gdn_layer_fwd(ctypes.byref(w), ctypes.byref(cfg), null, null, null, null, null, 0, null) == 6
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of the ABI structs have the C compiler's sizes and
+    field offsets (a C program including include/gdn.h prints them)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    mirrors = {"gdn_nvfp4_t": _lib.Nvfp4, "gdn_epilogue_segment_t": _lib.Segment,
+               "gdn_layer_cfg_t": _lib.LayerCfg, "gdn_layer_weights_t": _lib.LayerWeights}
+    lines = ["#include <stddef.h>", "#include <stdio.h>", '#include "gdn.h"', "int main(void) {"]
+    for cname, py in mirrors.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, py in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
