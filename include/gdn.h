@@ -226,6 +226,9 @@ int gdn_gates(const float* a, const float* b, int64_t M, int H,
  * GDN_DR_MMA_SYNC, run the warp-level mma.sync kernel.  Both compute the same
  * chunk form; they differ in FP32 summation order only.
  * ws     gdn_delta_rule_workspace_size(...) bytes (may be 0 / NULL).
+ * flags  GDN_DR_L2NORM_QK | GDN_DR_O_FP32 | GDN_DR_MMA_SYNC; any other bit
+ *        (GDN_DR_DECAYED_READ included: the chunked form implements the
+ *        literal read) is GDN_ERR_INVALID_ARG.
  * ------------------------------------------------------------------------ */
 enum { GDN_DR_L2NORM_QK = 1, GDN_DR_O_FP32 = 2, GDN_DR_MMA_SYNC = 4 };
 
