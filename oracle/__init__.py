@@ -28,9 +28,11 @@ Modules
   delta_rule  sequential gated delta rule (the literal recurrence) and the
               chunked (UT / WY) form, both FP64
   layer       the four steps composed into one layer forward
+  replay      clean vs NVFP4 trajectories of the recurrent state and the
+              decay of an impulse (the pages' robustness measurements)
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
-against closed forms, brute force or independent library routines; none is
-"parity unpinned" except the replay statistics, which the oracle does not
-define.
+against closed forms, brute force or independent library routines.  The
+values the replay harness reports are "parity unpinned": the pages' figures
+come from trained layers and real text; the harness itself is pinned.
 """

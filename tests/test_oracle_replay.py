@@ -1,0 +1,63 @@
+"""Pins of the replay harness (oracle/replay.py), CPU only.
+
+The statistics it reports (state error of NVFP4 trajectories against a clean
+one, impulse decay) have no values on the pages that synthetic inputs could
+reproduce; these tests pin the harness itself: it measures zero when nothing
+is quantized, the clean projections do not depend on the d_model permutation
+that makes the NVFP4 realisations independent, and an impulse on a
+write-free (beta = 0) trajectory decays exactly as the product of the decays.
+"""
+import numpy as np
+
+from nvfp4_w4a4_gated_quant_b200 import inputs
+from oracle.replay import clean_projections, impulse_response, replay
+
+D = dict(B=1, T=256, d_model=128, H=2, dk=32, dv=32)
+CHECK = (64, 128, 256)
+
+
+def _inputs():
+    return inputs.layer_inputs(D["B"], D["T"], D["d_model"], D["H"], D["dk"], D["dv"], seed=40)
+
+
+def test_no_quantization_means_no_state_error():
+    r = replay(_inputs(), seeds=(1, 2), checkpoints=CHECK, t_imp=128, window=16, quantize=False)
+    assert np.all(r["state_error"] < 1e-12)
+
+
+def test_clean_projections_do_not_depend_on_the_permutation():
+    d = _inputs()
+    x = d["x"].reshape(-1, D["d_model"])
+    perm = np.random.default_rng(7).permutation(D["d_model"])
+    p0 = clean_projections(x, d["W"])
+    p1 = clean_projections(x[:, perm], {n: np.asarray(d["W"][n])[:, perm] for n in ("q", "k", "v", "a", "b")})
+    for n in ("a", "b"):
+        np.testing.assert_allclose(p1[n], p0[n], rtol=1e-12, atol=1e-14)
+    for n in ("q", "k", "v"):
+        assert np.mean(p1[n] != p0[n]) < 1e-3          # bf16 rounding ties only
+
+
+def test_nvfp4_realisations_are_independent_and_bounded():
+    r = replay(_inputs(), seeds=(1, 2, 3), checkpoints=CHECK, t_imp=128, window=16)
+    e = r["state_error"]                                # [seeds, checkpoints]
+    assert e.shape == (3, len(CHECK))
+    assert np.all(np.isfinite(e)) and np.all(e > 1e-4) and np.all(e < 1.0)
+    assert len(set(np.round(e[:, -1], 12))) == 3        # three different realisations
+    np.testing.assert_allclose(r["mean"], e.mean(axis=0))
+    assert np.all(r["max"] >= r["mean"])
+
+
+def test_impulse_without_writes_decays_as_the_gate_product():
+    rng = np.random.default_rng(3)
+    B, T, H, dk, dv = 1, 96, 3, 8, 6
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk))
+    v = rng.standard_normal((B, T, H, dv))
+    la = rng.uniform(-0.3, -0.01, (B, T, H))
+    be = np.zeros((B, T, H))
+    # a nonzero state to perturb: writes before the impulse, none after it
+    be[:, :32] = 0.5
+    steps, horizon = impulse_response(q, k, v, la, be, t_imp=32, window=60, eps=0.01,
+                                      rng=np.random.default_rng(0))
+    assert np.all(horizon > 0)
+    np.testing.assert_array_equal(steps, horizon)
