@@ -7,11 +7,14 @@ trajectory with the states of NVFP4 trajectories over long sequences (a state
 error of a few tens of percent that does not grow without bound) and follow
 an impulse added to the state until it has decayed.  Their numbers come from
 trained layers and real text; here the same measurements run on synthetic
-inputs, so the statistics themselves are parity unpinned.  What is pinned
-(``tests/test_oracle_replay.py``) is the harness: zero error when nothing is
-quantized, the exact permutation invariance of the clean projections, and the
-impulse of a write-free (beta = 0) trajectory decaying exactly as the product
-of the decays.
+inputs, so the statistics themselves are parity unpinned.  The same page
+applies multiplicative noise directly to the gates (alpha and beta) to show
+where the recurrence is fragile; ``gate_noise_arm`` does that here.  What is
+pinned (``tests/test_oracle_replay.py``) is the harness: zero error when
+nothing is quantized or no noise is added, the exact permutation invariance
+of the clean projections, an impulse on a write-free (beta = 0) trajectory
+decaying exactly as the product of the decays, and alpha noise on such a
+trajectory scaling each head's state by exactly prod (1 + sigma z).
 
 Readings where the pages are silent:
   * clean trajectory: FP64 projections of the bf16 activations with the FP32
@@ -132,3 +135,29 @@ def replay(d, seeds, checkpoints, t_imp, window, eps=0.01, quantize=True):
     steps, horizon = impulse_response(*clean, t_imp, window, eps, np.random.default_rng(12345))
     return {"checkpoints": list(checkpoints), "state_error": errs, "mean": errs.mean(axis=0),
             "max": errs.max(axis=0), "impulse_steps": steps, "decay_horizon": horizon}
+
+
+def gate_noise_arm(scan_in, sigma, target, seeds, checkpoints, S0=None):
+    """Multiplicative gate noise on a given trajectory: every alpha_t (target
+    "alpha") or beta_t ("beta") times (1 + sigma z), z ~ N(0, 1) per (token,
+    head), seeded.  Returns the relative state error against the noise-free
+    trajectory, [seeds, checkpoints]."""
+    q, k, v, la, be = scan_in
+    S_ref = states_at(q, k, v, la, be, checkpoints, S0=S0)
+    out = []
+    for s in seeds:
+        z = np.random.default_rng(s).standard_normal(la.shape)
+        f = 1.0 + sigma * z
+        assert np.all(f > 0), "noise too large for a multiplicative perturbation"
+        la_n, be_n = (la + np.log(f), be) if target == "alpha" else (la, be * f)
+        S_n = states_at(q, k, v, la_n, be_n, checkpoints, S0=S0)
+        out.append([rel_state_error(a, b) for a, b in zip(S_n, S_ref)])
+    return np.asarray(out)
+
+
+def clean_scan_inputs(d):
+    """The clean trajectory's scan inputs (q, k, v, log_alpha, beta) for the
+    layer inputs ``d``."""
+    B, T, D, H, dk, dv = d["B"], d["T"], d["d_model"], d["H"], d["dk"], d["dv"]
+    return _scan_inputs(clean_projections(d["x"].reshape(B * T, D), d["W"]), B, T, H, dk, dv, d["A_log"],
+                        d["dt_bias"])

@@ -61,3 +61,30 @@ def test_impulse_without_writes_decays_as_the_gate_product():
                                       rng=np.random.default_rng(0))
     assert np.all(horizon > 0)
     np.testing.assert_array_equal(steps, horizon)
+
+
+def test_gate_noise_arm_zero_noise_and_write_free_closed_form():
+    from oracle.replay import clean_scan_inputs, gate_noise_arm
+    scan_in = clean_scan_inputs(_inputs())
+    assert np.all(gate_noise_arm(scan_in, 0.0, "alpha", (1, 2), CHECK) == 0.0)
+    assert np.all(gate_noise_arm(scan_in, 0.0, "beta", (1, 2), CHECK) == 0.0)
+    # write-free trajectory from a nonzero state: S_t = prod(alpha) S_0, so
+    # alpha noise scales head h's state by prod_s (1 + sigma z_s) exactly
+    rng = np.random.default_rng(5)
+    B, T, H, dk, dv = 1, 40, 3, 6, 4
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk))
+    v = rng.standard_normal((B, T, H, dv))
+    la = rng.uniform(-0.2, -0.01, (B, T, H))
+    be = np.zeros((B, T, H))
+    S0 = rng.standard_normal((B, H, dk, dv))
+    sigma = 0.01
+    e = gate_noise_arm((q, k, v, la, be), sigma, "alpha", (9,), (T,), S0=S0)
+    z = np.random.default_rng(9).standard_normal(la.shape)
+    g = np.prod(1.0 + sigma * z, axis=1)                         # [B, H]
+    n2 = np.sum(S0 ** 2, axis=(2, 3))                            # ||S0_h||^2
+    G = np.exp(np.sum(la, axis=1))
+    want = np.sqrt(np.sum((G * (g - 1.0)) ** 2 * n2) / np.sum(G ** 2 * n2))
+    np.testing.assert_allclose(e[0, 0], want, rtol=1e-9)
+    # beta noise cannot act without writes
+    assert np.all(gate_noise_arm((q, k, v, la, be), sigma, "beta", (9,), (T,), S0=S0) == 0.0)
