@@ -338,12 +338,13 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg,
 /* ------------------------------------------------------------------------ *
  * Allocation-free layer forward (no counterpart in the paper).
  *
- * For callers that cannot allocate device memory: code running while a CUDA
- * graph is being captured without an allocator, plugins that receive only
- * their input and output pointers, real-time paths with a fixed memory budget.
- * Same computation, arguments and results as gdn_layer_fwd, except that the
- * workspace is a static device array of GDN_LAYER_STATIC_WS_BYTES inside the
- * library (present on every GPU that loads it, until the process exits).
+ * For callers that cannot allocate device memory: plugins that receive only
+ * their input and output pointers from a host framework that owns every
+ * allocation, and real-time paths whose memory budget is fixed up front.
+ * Same computation, arguments and results as gdn_layer_fwd (bit for bit),
+ * except that the workspace is a static device array of
+ * GDN_LAYER_STATIC_WS_BYTES inside the library (present on every GPU that
+ * loads it, until the process exits).
  *   - Sizes: a cfg whose gdn_layer_workspace_size() exceeds the array is
  *     rejected with GDN_ERR_WORKSPACE (gdn_last_error() says by how much);
  *     with d_model 5120, H 32, d 128 that is about 860 tokens per call.
@@ -354,6 +355,10 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg,
  *     the GPU (different streams, or threads without ordering) race; order
  *     them on one stream.  The array keeps the last call's intermediates.
  *   - Allocates nothing: no cudaMalloc / cudaFree or allocating routine.
+ *   - The looked-up address is cached per device for the life of the
+ *     process: do not call this entry point again after cudaDeviceReset()
+ *     (or any other teardown of the device's primary context).  The same
+ *     holds for the device status word every entry point writes.
  * ------------------------------------------------------------------------ */
 #define GDN_LAYER_STATIC_WS_BYTES (32u << 20)
 

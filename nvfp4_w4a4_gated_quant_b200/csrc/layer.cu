@@ -140,12 +140,12 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
 // ---------------------------------------------------------------------------
 // Allocation-free layer forward.
 //
-// Some callers cannot allocate device memory at all: code that runs while a
-// CUDA graph is being captured with no allocator to hand, plugins that are
-// given only their input and output pointers, and real-time paths whose
-// memory budget is fixed up front.  They call gdn_layer_fwd_static_ws, which
-// takes the layer's scratch (the intermediates between its kernels) from the
-// file-scope device array below instead of a caller workspace.
+// Some callers cannot allocate device memory at all: plugins that are given
+// only their input and output pointers by a host framework that owns every
+// allocation, and real-time paths whose memory budget is fixed up front.  They
+// call gdn_layer_fwd_static_ws, which takes the layer's scratch (the
+// intermediates between its kernels) from the file-scope device array below
+// instead of a caller workspace.
 //
 // The array is GDN_LAYER_STATIC_WS_BYTES (32 MiB) and lives on every GPU that
 // loads this library until the process exits.  Host code cannot pass the

@@ -120,3 +120,11 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_static_scratch_size_matches_header():
+    """The binding's copy of the static scratch size is the header's."""
+    text = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    m = re.search(r"#define\s+GDN_LAYER_STATIC_WS_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m, "GDN_LAYER_STATIC_WS_BYTES not found in gdn.h"
+    assert _lib.LAYER_STATIC_WS_BYTES == int(m.group(1)) << int(m.group(2))

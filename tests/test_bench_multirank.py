@@ -69,3 +69,30 @@ def test_two_rank_timing_and_aggregation():
         assert value == pytest.approx(2 * 32768 / 0.013)   # all ranks' tokens over the slowest time
     assert res[0][5] != res[1][5]                          # independent batches per rank
     assert res[1][6] is None                               # the reference arm runs on rank 0 only
+
+
+def test_launch_plan():
+    import bench
+    assert bench.launch_plan(None, {}) == ("run", 1)
+    assert bench.launch_plan(1, {}) == ("run", 1)
+    assert bench.launch_plan(4, {}) == ("relaunch", 4)
+    assert bench.launch_plan(None, {"WORLD_SIZE": "2"}) == ("run", 2)
+    assert bench.launch_plan(2, {"WORLD_SIZE": "2"}) == ("run", 2)
+    assert bench.launch_plan(8, {"WORLD_SIZE": "2"})[0] == "error"
+    assert bench.launch_plan(0, {})[0] == "error"
+
+
+def test_gpus_flag_runs_that_many_ranks():
+    """`bench.py --gpus 2` outside a launcher starts two ranks under
+    torch.distributed.run; the reference arm (CPU, rank 0 alone) then reports
+    n_gpus 2.  (The other arm needs CUDA devices.)"""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0", "--sample-tokens", "16"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2

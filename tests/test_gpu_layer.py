@@ -5,8 +5,10 @@ Each stage is compared with the oracle fed the GPU's own inputs to that stage
 own: x and o codes / scales bit-exact, projections 1e-3 (bf16 vs bf16), gates
 1e-4, o 3e-3 (bf16 storage), y 1e-3.  End to end, with every stage's error
 compounding through 4-bit requantisation of o, y is compared with the fully
-independent oracle layer at 5e-2 relative Frobenius (4-bit codes of o flip at
-rounding boundaries when o moves by its bf16 error).
+independent oracle layer at 1e-2 relative Frobenius (4-bit codes of o flip at
+rounding boundaries when o moves by its bf16 error; measured 5.5e-3 on the
+tiny layer) and the final state at 2e-3, the scan's own tolerance (measured
+3.0e-4).
 """
 import numpy as np
 import pytest
@@ -102,8 +104,8 @@ def test_tiny_layer_stagewise_and_end_to_end():
     y_ref, S_ref2, _ = layer_forward(d["x"], Wq, d["A_log"], d["dt_bias"], H, dk, dv)
     e2e = rel_fro(y_gpu, y_ref.reshape(M, D))
     print(f"tiny layer end-to-end rel_fro {e2e:.3e}")
-    assert e2e < 5e-2
-    assert rel_fro(to_np(S_T), S_ref2) < 2e-2
+    assert e2e < 1e-2
+    assert rel_fro(to_np(S_T), S_ref2) < 2e-3
 
 
 def test_layer_workload_sampled():
