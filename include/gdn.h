@@ -58,7 +58,10 @@ typedef enum {
   GDN_ERR_ALIGNMENT = 3,         /* a pointer or stride breaks an alignment rule */
   GDN_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed         */
   GDN_ERR_TIMEOUT = 5,           /* a bounded device-side wait ran out          */
-  GDN_ERR_WORKSPACE = 6          /* workspace missing or smaller than required  */
+  GDN_ERR_WORKSPACE = 6,         /* workspace missing or smaller than required  */
+  GDN_ERR_RANGE = 7              /* a value left the FP16 range of the scan's
+                                    tensor-core operands (|x| >= 65520); the
+                                    outputs of that call are not valid          */
 } gdn_status_t;
 
 typedef void* gdn_stream_t; /* cudaStream_t */
@@ -218,9 +221,15 @@ int gdn_gates(const float* a, const float* b, int64_t M, int H,
  * o      [B, T, H, dv] contiguous; bf16, or FP32 with GDN_DR_O_FP32.
  * S_T    FP32 [B, H, dk, dv] final state, or NULL.
  * Supported: dk and dv in {32, 64, 128}; any T >= 0 (a ragged last chunk is
- * handled); B*H >= 1.  Values of v and of the state must stay inside the
- * FP16 range (|x| < 65504): the chunk contractions run on FP16 tensor-core
- * operands with FP32 accumulation.
+ * handled); B*H >= 1.  The chunk contractions run on FP16 tensor-core
+ * operands with FP32 accumulation (FP16 keeps three more mantissa bits than
+ * bf16, which the 2e-3 tolerance at 32K tokens needs).  Values of beta v, of
+ * the state and of the chunk intermediates must stay inside the FP16 range:
+ * a value of magnitude >= 65520 rounds to infinity, and the call then records
+ * GDN_ERR_RANGE in the device status word (gdn_stream_check() returns it);
+ * its o and S_T are not valid.  With the tensor-core kernel every FP16
+ * operand is checked where it is converted; with the mma.sync kernel the
+ * check is that o and S_T came out finite.
  * Kernels: dk = 128 with dv a multiple of 64 runs on the 5th-generation
  * tensor cores (tcgen05.mma, state kept in TMEM); other shapes, or the flag
  * GDN_DR_MMA_SYNC, run the warp-level mma.sync kernel.  Both compute the same

@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgdn.so")
 
 GDN_OK = 0
+ERR_TIMEOUT, ERR_WORKSPACE, ERR_RANGE = 5, 6, 7
 QUANT_DYNAMIC, QUANT_GIVEN_SCALE, QUANT_GIVEN_AMAX = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
 SF_TILED, SF_LINEAR = 0, 1
@@ -111,7 +112,7 @@ def check(status):
     if status != GDN_OK:
         L = lib()
         msg = L.gdn_status_string(status).decode()
-        if status == 4:
+        if status in (4, 6):
             msg += ": " + L.gdn_last_error().decode()
         raise GdnError(f"gdn status {status}: {msg}")
 

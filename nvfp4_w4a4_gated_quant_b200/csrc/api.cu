@@ -142,6 +142,7 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_CUDA: return "CUDA error";
     case GDN_ERR_TIMEOUT: return "device-side wait timed out";
     case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    case GDN_ERR_RANGE: return "a scan operand left the FP16 range";
     default: return "unknown status";
   }
 }

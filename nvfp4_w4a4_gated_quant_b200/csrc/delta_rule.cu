@@ -164,6 +164,7 @@ struct Args {
   void* o;
   float* S_T;
   unsigned* o_amax;   // optional: FP32 bits of max |stored o| (atomicMax), for the next quantizer
+  int* status;        // device status word (GDN_ERR_RANGE when an output is not finite)
 };
 
 template <int DK, int DVS>
@@ -709,6 +710,18 @@ __global__ void __launch_bounds__(NT, 1) delta_rule_kernel(const __grid_constant
     __syncthreads();
   }
 
+  // An FP16 operand that overflowed (|x| >= 65520 rounds to infinity) reaches
+  // o or the FP32 state as inf or NaN: report it instead of returning it silently.
+  {
+    bool bad = amax_bits >= 0x7F800000u;
+    if (s_owner) {
+#pragma unroll
+      for (int j = 0; j < NVT; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bad |= !isfinite(S[j][e]);
+    }
+    if (bad) report_status(a.status, GDN_ERR_RANGE);
+  }
   if (a.o_amax) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax_bits = max(amax_bits, __shfl_xor_sync(0xffffffffu, amax_bits, o));
@@ -788,6 +801,7 @@ int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, i
   a.o = o;
   a.S_T = S_T;
   a.o_amax = o_amax;
+  a.status = device_status_word();
   const bool f32 = (flags & GDN_DR_O_FP32) != 0;
   switch (dk) {
     case 32: return f32 ? launch_dk<32, true>(a, dvs, chains, stream) : launch_dk<32, false>(a, dvs, chains, stream);

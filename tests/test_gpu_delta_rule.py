@@ -121,3 +121,24 @@ def test_delta_rule_strong_and_no_decay():
             o, S = _run(q, k, v, la, be, S0, mma_sync=mma_sync)
             assert np.isfinite(o).all() and np.isfinite(S).all()
             assert rel_fro(o, o_ref) < TOL and rel_fro(S, S_ref) < TOL, (la_val, mma_sync)
+
+
+@pytest.mark.parametrize("mma_sync", [False, True], ids=["tcgen05", "mma_sync"])
+def test_fp16_overflow_is_reported(mma_sync):
+    """A value of v beyond the FP16 range of the chunk contractions
+    (|beta v| >= 65520 rounds to infinity) makes the call report
+    GDN_ERR_RANGE through the status word instead of returning inf / NaN
+    silently; the next call on the same context is unaffected."""
+    q, k, v, la, be, _ = _case(1, 100, 2, 128, 128, 11)
+    v = v.copy()
+    v[0, 37, 1, 5] = 2.0 ** 17
+    be = np.ones_like(be)
+    _lib.gdn_delta_rule_fwd(bf16_cuda(q), bf16_cuda(k), bf16_cuda(v), f32_cuda(la), f32_cuda(be), o_fp32=True,
+                            mma_sync=mma_sync)
+    with pytest.raises(_lib.GdnError, match="status 7"):
+        _lib.stream_check()
+    _lib.stream_check()      # the status word was cleared
+    q, k, v, la, be, S0 = _case(1, 100, 2, 128, 128, 12)
+    o, S = _run(q, k, v, la, be, S0, mma_sync=mma_sync)
+    o_ref, S_ref = delta_rule_chunked(q, k, v, la, be)
+    assert rel_fro(o, o_ref) < TOL and rel_fro(S, S_ref) < TOL
