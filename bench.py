@@ -273,10 +273,11 @@ def run_ours(args, rank, world, local_rank):
     stage_ms = {name: statistics.mean(sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(args.steps))
                 for j, (name, _) in enumerate(stages)}
 
-    # ---- the layer with a static encode scale for o (its NVFP4 quantization
-    # done in the scan's epilogue, no o quantizer pass).  The scale is this
-    # input's own dynamic one, so the layer's output is the same.
-    lw.o_g_enc = (torch.full((1,), 2688.0, dtype=torch.float32, device=dev) / o_amax).contiguous()
+    # ---- the layer with static, per-module calibrated activation scales: x
+    # quantized in one pass (no amax pass), o quantized in the scan's epilogue
+    # (no quantizer pass).  Calibrated on this input itself, so the scales are
+    # its dynamic ones and the layer's output is the same.
+    lw.x_g_enc, lw.o_g_enc = _lib.calibrate_layer(lw, [x])
     for _ in range(args.warmup):
         layer_step()
     ss0, ss1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -289,9 +290,35 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     _lib.stream_check()
-    lw.o_g_enc = None
+    lw.x_g_enc = lw.o_g_enc = None
     static_ms = max_over_ranks(ss0.elapsed_time(ss1), world, dev)
     static_value, static_ms_step = aggregate(static_ms, args.steps, M, world)
+
+    # ---- the layer with the rest of a Gated DeltaNet block (outside
+    # specification): a sixth W4A4 projection g, the short convolution + SiLU
+    # on q, k, v and the gated RMSNorm of o (seeded synthetic weights)
+    rng_ext = np.random.default_rng(replica_seed(rank) + 100)
+    W_ext = dict(d["W"])
+    W_ext["g"] = inputs.weight(rng_ext, HV, D)
+    lw_ext = _lib.QuantizedLayerWeights(W_ext, d["A_log"], d["dt_bias"], H, dk, dv, device=dev,
+                                        conv_w=rng_ext.uniform(-0.6, 0.6, (2 * HK + HV, 4)).astype(np.float32),
+                                        norm_w=rng_ext.uniform(0.5, 1.5, dv).astype(np.float32))
+    ws_ext = torch.empty(_lib.gdn_layer_workspace_size(lw_ext.cfg(B, T)), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        _lib.gdn_layer_fwd(lw_ext, x, y=y, S_T=S_T, ws=ws_ext)
+    ex0, ex1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ex0.record(stream)
+    for _ in range(args.steps):
+        _lib.gdn_layer_fwd(lw_ext, x, y=y, S_T=S_T, ws=ws_ext)
+    ex1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    _lib.stream_check()
+    ext_ms = max_over_ranks(ex0.elapsed_time(ex1), world, dev)
+    ext_value, ext_ms_step = aggregate(ext_ms, args.steps, M, world)
+    del lw_ext, ws_ext
 
     # ---- end to end through the public call with host buffers: every step
     # copies its input in from pinned host memory and its output back, with
@@ -333,9 +360,11 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.summary()
     tokens_per_step = M * world
     pk = peaks()
-    # FP4 dense = 4x bf16 (the nominal 9 / 2.25 PFLOP/s ratio) on the measured
-    # burst bf16 rate: the layer step is milliseconds long, not a sustained run
-    fp4_peak = 4.0 * pk["bf16_tflops"]
+    # the FP4 denominator: the tensor pipe's own ceiling for this MMA, measured
+    # on this GPU in this run; without it, 4x the measured burst bf16 rate (the
+    # nominal 9 / 2.25 PFLOP/s ratio)
+    fp4_ceiling = kernels.get("fp4_mma_ceiling", {}).get("TFLOPs") if kernels else None
+    fp4_peak = fp4_ceiling or 4.0 * pk["bf16_tflops"]
     costs = stage_costs(B, T, D, H, dk, dv)
     stage_out = {}
     for name, ms in stage_ms.items():
@@ -361,8 +390,9 @@ def run_ours(args, rank, world, local_rank):
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["traffic"] = traffic_from_profiles(dom)
     roof["kernel"] = f"{dom} ({kname})"
-    roof["peak_source"] = (f"{pk['source']}: " + ("hbm_gbs" if bound == "hbm" else
-                                                  "4 x bf16_tflops burst (FP4 = 4x bf16 nominal)"))
+    roof["peak_source"] = (f"{pk['source']}: hbm_gbs" if bound == "hbm" else
+                           "measured in this run: gdn_fp4_mma_ceiling" if fp4_ceiling else
+                           f"{pk['source']}: 4 x bf16_tflops burst (FP4 = 4x bf16 nominal)")
     if bound == "tensor":
         roof["frac_fp4_nominal_9PF"] = round(roof["achieved"] / 9000.0, 4)
 
@@ -379,9 +409,13 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": LAUNCHES_PER_LAYER_STEP * args.steps,
         "roofline": roof,
         "stages": stage_out,
-        "static_o_scale": {"value": round(static_value, 1), "unit": UNIT, "ms_per_step": round(static_ms_step, 4),
-                           "what": "the same layer with a static encode scale for o (equal to this input's "
-                                   "dynamic one): o quantized in the scan epilogue, no o quantizer pass"},
+        "static_scales": {"value": round(static_value, 1), "unit": UNIT, "ms_per_step": round(static_ms_step, 4),
+                          "what": "the same layer with per-module calibrated static activation scales (x and o, "
+                                  "calibrated on this input, so equal to its dynamic ones): x quantized in one "
+                                  "pass, o quantized in the scan epilogue"},
+        "with_conv_and_out_gate": {"value": round(ext_value, 1), "unit": UNIT, "ms_per_step": round(ext_ms_step, 4),
+                                   "what": "the layer with a sixth projection g (H*dv more GEMM columns), the short "
+                                           "convolution + SiLU on q/k/v and the gated RMSNorm of o"},
         "clocks": clk,
         "step_ms_min_max": [round(min(step_ms), 4), round(max(step_ms), 4)],
     }
@@ -390,6 +424,23 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.skip_cpu:
         line["cpu_baseline"] = cpu_baseline(seconds_budget=args.cpu_seconds, T_sample=args.sample_tokens)
     return line
+
+
+def fp4_ceiling_tflops(torch, _lib, stream, iters=40000, reps=3):
+    """The FP4 tensor-core ceiling of the GEMM's MMA (gdn_fp4_mma_ceiling:
+    one CTA per SM issuing 128 x 256 x 64 block-scaled MMAs back to back from
+    resident operands), best of `reps` runs of ~20 ms, in TFLOP/s."""
+    best = 0.0
+    _lib.fp4_mma_ceiling(1000, stream)
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        flops = _lib.fp4_mma_ceiling(iters, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = max(best, flops / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    _lib.stream_check()
+    return best
 
 
 def standalone_kernels(args, torch, _lib, inputs, dev, stream, which=None):
@@ -418,7 +469,12 @@ def standalone_kernels(args, torch, _lib, inputs, dev, stream, which=None):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     tf = 2.0 * M * N * K / (ms / 1e3) / 1e12
+    ceil = fp4_ceiling_tflops(torch, _lib, stream)
+    out["fp4_mma_ceiling"] = {"TFLOPs": round(ceil, 1), "what": "gdn_fp4_mma_ceiling: 128x256x64 mxf4nvf4 MMAs "
+                                                               "back to back from resident operands, one CTA per SM",
+                              "frac_fp4_nominal_9PF": round(ceil / 9000.0, 4)}
     out["gemm_8192x12288x5120"] = {"us": round(ms * 1e3, 1), "TFLOPs": round(tf, 1),
+                                   "frac_fp4_ceiling": round(tf / ceil, 4),
                                    "frac_fp4_burst": round(tf / (4 * pk["bf16_tflops"]), 4),
                                    "frac_fp4_nominal_9PF": round(tf / 9000.0, 4)}
     del x, w, xc, xs, wc, wsc, y
@@ -560,6 +616,85 @@ def run_reference(args, rank, world):
     }
 
 
+# --------------------------------------------------------- replay workload --
+REPLAY = dict(B=1, T=32768, d_model=5120, H=16, dk=128, dv=128, seed=4, checkpoints=(256, 4096, 32768),
+              seeds=tuple(range(1, 12)), t_imp=1024, window=2048, eps=0.01)
+
+
+def run_replay(args):
+    """The replay workload: the oracle's clean trajectory (FP64 projections of
+    the bf16 activations, scan in FP64) on the host, and 11 NVFP4
+    trajectories (independent d_model permutations) through the library;
+    relative state error at the checkpoints, the library's scan on the clean
+    inputs (its own error), an impulse of 1% at token 1024 followed through
+    the library's decode step, and the gate-error compression (projection
+    error on a / b against the error on 1 - alpha and beta)."""
+    import torch
+    from nvfp4_w4a4_gated_quant_b200 import inputs, replay
+    from oracle import replay as oreplay
+    R = REPLAY
+    T, Dm, H, dk, dv = R["T"], R["d_model"], R["H"], R["dk"], R["dv"]
+    t_start = time.perf_counter()
+    d = inputs.layer_inputs(R["B"], T, Dm, H, dk, dv, seed=R["seed"])
+    x = d["x"].reshape(T, Dm)
+    _all_host_threads()
+    t0 = time.perf_counter()
+    clean_proj = oreplay.clean_projections(x, d["W"])
+    clean = oreplay._scan_inputs(clean_proj, 1, T, H, dk, dv, d["A_log"], d["dt_bias"])
+    S_clean = oreplay.states_at(*clean, R["checkpoints"])
+    oracle_s = time.perf_counter() - t0
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    # the library's own error: its scan on the clean inputs
+    cd = (torch.from_numpy(clean[0].astype(np.float32)).to(dev).to(torch.bfloat16),
+          torch.from_numpy(clean[1].astype(np.float32)).to(dev).to(torch.bfloat16),
+          torch.from_numpy(clean[2].astype(np.float32)).to(dev).to(torch.bfloat16),
+          torch.from_numpy(clean[3].astype(np.float32)).to(dev).contiguous(),
+          torch.from_numpy(clean[4].astype(np.float32)).to(dev).contiguous())
+    eps0 = [oreplay.rel_state_error(a.cpu().numpy(), b) for a, b in zip(replay.states_at(*cd, R["checkpoints"]),
+                                                                       S_clean)]
+    errs, gate = [], []
+    steps_q = None
+    for sd in R["seeds"]:
+        perm = np.random.default_rng(sd).permutation(Dm)
+        qkv, a, b = replay.nvfp4_projections(x, d["W"], H, dk, dv, perm=perm, device=dev)
+        sin = replay.scan_inputs(qkv, a, b, d["A_log"], d["dt_bias"], T, H, dk, dv)
+        S_q = replay.states_at(*sin, R["checkpoints"])
+        errs.append([oreplay.rel_state_error(sq.cpu().numpy(), sc) for sq, sc in zip(S_q, S_clean)])
+        g = oreplay.gate_error_compression(clean_proj["a"], clean_proj["b"], a.cpu().numpy().astype(np.float64),
+                                           b.cpu().numpy().astype(np.float64), d["A_log"], d["dt_bias"])
+        gate.append([g["a"], g["b"], g["one_minus_alpha"], g["beta"]])
+        if steps_q is None:
+            steps_q = replay.impulse_steps(*sin, R["t_imp"], R["window"], R["eps"], seed=12345)
+        del qkv, a, b, sin, S_q
+    errs = np.asarray(errs)
+    gate = np.asarray(gate)
+    # the clean trajectory's impulse (oracle, FP64) and its decay-implied horizon
+    steps_c, horizon = oreplay.impulse_response(*clean, R["t_imp"], min(R["window"], 256), R["eps"],
+                                                np.random.default_rng(12345))
+    return {
+        "impl": "ours", "mode": "replay",
+        "config": {"workload": f"replay B=1 x 12 trajectories T={T} d_model={Dm} H={H} dk=dv={dk} seed {R['seed']}",
+                   "checkpoints": list(R["checkpoints"]), "nvfp4_trajectories": len(R["seeds"]),
+                   "impulse": f"S *= 1 + {R['eps']} z at token {R['t_imp']}"},
+        "state_error": {"mean": [round(float(v), 4) for v in errs.mean(axis=0)],
+                        "max": [round(float(v), 4) for v in errs.max(axis=0)],
+                        "per_seed": [[round(float(v), 4) for v in row] for row in errs]},
+        "library_scan_error_on_clean_inputs": [float(f"{v:.3e}") for v in eps0],
+        "impulse_steps_to_1_over_e": {"nvfp4_library_per_head": steps_q.tolist(),
+                                      "clean_oracle_per_head": steps_c[0].tolist(),
+                                      "decay_horizon_per_head": horizon[0].tolist(),
+                                      "median_nvfp4_library": float(np.median(steps_q))},
+        "gate_error_compression": {"projection_a": round(float(gate[:, 0].mean()), 4),
+                                   "projection_b": round(float(gate[:, 1].mean()), 4),
+                                   "one_minus_alpha": round(float(gate[:, 2].mean()), 4),
+                                   "beta": round(float(gate[:, 3].mean()), 4)},
+        "oracle_seconds": round(oracle_s, 1), "host_threads": _threads(),
+        "wall_seconds": round(time.perf_counter() - t_start, 1),
+        "parity": "statistics unpinned (synthetic inputs); the path is pinned by tests/test_gpu_replay.py",
+    }
+
+
 def launch_plan(gpus, env):
     """How to run for ``--gpus`` (None: take the launcher's WORLD_SIZE) given
     the environment: ("run", world) in this process, ("relaunch", n) as n
@@ -606,6 +741,8 @@ def main():
                     help="tokens of the oracle sample (CPU baseline and --impl reference)")
     ap.add_argument("--only", choices=["gemm", "scan"], default=None,
                     help="time only the standalone GEMM or scan workload (profiling target)")
+    ap.add_argument("--replay", action="store_true",
+                    help="run the replay workload (state error of NVFP4 trajectories, impulse, gate errors)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -622,6 +759,9 @@ def main():
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return
+    if args.replay:
+        print(json.dumps(run_replay(args)), flush=True)
         return
     if args.only:
         import torch

@@ -83,6 +83,15 @@ int gdn_stream_check(gdn_stream_t stream);
  * watchdog path without faulting or hanging anything. */
 int gdn_selftest_bounded_wait(uint32_t poll_limit, gdn_stream_t stream);
 
+/* Diagnostic: the FP4 tensor-core ceiling of gdn_gemm_nvfp4's MMA.  Enqueues
+ * one CTA per SM (*ctas receives the count), each issuing iters x 4
+ * tcgen05.mma.kind::mxf4nvf4.block_scale.block16 of M = 128, N = 256, K = 64
+ * back to back from operands resident in shared memory and scales resident
+ * in TMEM (no loads, no epilogue): 2 * 128 * 256 * 64 * 4 * iters * *ctas
+ * FLOP.  Time it with events on `stream`; the achieved rate is the ceiling a
+ * GEMM of this shape is measured against.  iters in 1 .. 2^32. */
+int gdn_fp4_mma_ceiling(int64_t iters, int* ctas, gdn_stream_t stream);
+
 /* ------------------------------------------------------------------------ *
  * Step 1: quantize activations to NVFP4.
  *
@@ -132,6 +141,29 @@ int gdn_quantize_nvfp4(const void* x, int x_dtype, int64_t rows, int64_t cols, i
                        uint8_t* codes, uint8_t* scales, int sf_layout,
                        int64_t sf_row_offset, float* g_out,
                        void* ws, size_t ws_bytes, gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
+ * Calibration of static activation scales.
+ *
+ * Passage: "Why Gated DeltaNet Survives 4-Bit Quantization", section
+ * "Critical Lessons for Model Serving" -- activation scales are calibrated
+ * for each module on its own, and a fused module must keep every module's
+ * own scale.  A static scale is the encode scale of the largest |x| a module
+ * saw over a calibration set: run gdn_amax_update on every calibration batch
+ * of that module's input (one running amax per module), then
+ * gdn_encode_scale_from_amax.  gdn_layer_fwd takes the two activation
+ * scales of the layer, x_g_enc and o_g_enc (gdn_layer_weights_t).
+ *
+ * gdn_amax_update: *amax = max(*amax, max |x|) over x [rows, cols] (row
+ *   stride ld_x elements; bf16 or FP32; 16-byte aligned, cols % 16 == 0).
+ *   *amax is a device FP32, >= 0 on entry (zero it before the first batch);
+ *   it is never reset by the call.  rows == 0 leaves it unchanged.
+ * gdn_encode_scale_from_amax: *g_enc = 2688 / *amax in FP32 (1 for 0; FLT_MAX
+ *   when the quotient overflows), the encode scale step 1 uses; both device.
+ * ------------------------------------------------------------------------ */
+int gdn_amax_update(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, float* amax,
+                    gdn_stream_t stream);
+int gdn_encode_scale_from_amax(const float* amax, float* g_enc, gdn_stream_t stream);
 
 /* ------------------------------------------------------------------------ *
  * Step 2: block-scaled FP4 GEMM  Y[m, n] = sum_k A_hat[m, k] * B_hat[n, k].
@@ -283,19 +315,58 @@ int gdn_delta_rule_step(const void* q, const void* k, const void* v,
                         int flags, void* o, gdn_stream_t stream);
 
 /* ------------------------------------------------------------------------ *
+ * The rest of a Gated DeltaNet block: short convolution and gated output norm.
+ *
+ * The pages name "the convolution" only as an alternative explanation and
+ * define neither piece; both follow the outside specification of the Gated
+ * DeltaNet block (Yang, Kautz and Hatamizadeh, "Gated Delta Networks:
+ * Improving Mamba2 with Delta Rule", ICLR 2025).
+ *
+ * gdn_short_conv: causal depthwise convolution of width 4 over tokens, then
+ *   SiLU, per channel c of x [B, T, C] (bf16, row stride ld_x elements):
+ *     y_t[c] = SiLU(sum_{j=0..3} w[c*4 + j] * x_{t-3+j}[c]),   SiLU(u) = u sigmoid(u)
+ *   w FP32 [C, 4] (16-byte aligned).  Tokens before t = 0 come from state_in
+ *   (bf16 [B, 3, C], the last three inputs of the previous call, oldest
+ *   first) or are zero when it is NULL; state_out (bf16 [B, 3, C], may be
+ *   NULL) receives this call's last three inputs, carried state included.
+ *   y bf16 [B, T, C] with row stride ld_y; must not alias x.  C % 8 == 0,
+ *   x, y 16-byte aligned, ld % 8 == 0; B <= 65535, T <= 65535 * 64.  FP32
+ *   arithmetic, CUDA's expf.
+ * gdn_gated_rmsnorm: per (token m, head h) row of dv values of o and g
+ *   (bf16 [M, H*dv], row m*H + h at (m*H + h)*dv):
+ *     y = o / sqrt(mean(o^2) + 1e-6) * gamma * SiLU(g)          (bf16 out)
+ *   gamma FP32 [dv]; dv in {32, 64, 128}.  When amax is non-NULL, max |y|
+ *   (of the stored bf16 values) is folded into *amax (>= 0 on entry), for a
+ *   given-amax quantization of y.
+ * ------------------------------------------------------------------------ */
+int gdn_short_conv(const void* x, int64_t B, int64_t T, int64_t C, int64_t ld_x, const float* w, const void* state_in,
+                   void* y, int64_t ld_y, void* state_out, gdn_stream_t stream);
+int gdn_gated_rmsnorm(const void* o, const void* g, int64_t M, int H, int dv, const float* gamma, void* y,
+                      float* amax, gdn_stream_t stream);
+
+/* ------------------------------------------------------------------------ *
  * The layer: steps 1-4 and the output projection, in one call.
  *
  *   xq = quant(x); [q|k|v|a|b] = gemm(xq, W_qkvab) with gates in the epilogue;
  *   o  = delta_rule(q, k, v, log_alpha, beta; L2-normalised q, k);
- *   y  = gemm(quant(o), W_out)  (bf16 out); quant(o) uses o's own amax, or
- *        the static encode scale w->o_g_enc when one is given.
- * No short convolution, output gate, norm or residual.
+ *   y  = gemm(quant(o), W_out)  (bf16 out); quant(x) and quant(o) use their
+ *        tensor's own amax, or the static encode scales w->x_g_enc and
+ *        w->o_g_enc when they are given (calibrated per module, see
+ *        "Calibration of static activation scales").
+ * Optional (cfg->conv, cfg->out_gate), from the Gated DeltaNet block's outside
+ * specification: q, k, v pass through gdn_short_conv (zero history: each
+ * call holds whole sequences) before the scan, and o through
+ * gdn_gated_rmsnorm with g = x W_g (a sixth W4A4 projection) before it is
+ * quantized for the output projection.  No residual.
  *
  * Weights are pre-quantized by the caller (gdn_quantize_nvfp4, one call per
  * projection so each keeps its own decode scale; q, k, v, a, b share one TILED
  * scale buffer through sf_row_offset).  W_qkvab rows: q [0, H*dk), k [H*dk,
  * 2*H*dk), v [2*H*dk, 2*H*dk + H*dv), a (H rows), b (H rows); K = d_model.
- * W_out: [d_model, H*dv].
+ * W_out: [d_model, H*dv].  With cfg->out_gate, W_qkvab holds H*dv more rows
+ * after b: the output gate g (decode scale w->g_g), and w->norm_w is the
+ * RMSNorm weight [dv]; with cfg->conv, w->conv_w is the convolution weight
+ * FP32 [2*H*dk + H*dv, 4] over the q | k | v channels.
  *
  * x   bf16 [B*T, d_model];  y bf16 [B*T, d_model];  S0 / S_T as in step 4.
  * ws  gdn_layer_workspace_size(cfg) bytes, 256-byte aligned.  After the call
@@ -306,6 +377,8 @@ int gdn_delta_rule_step(const void* q, const void* k, const void* v,
 typedef struct {
   int64_t B, T, d_model;
   int H, dk, dv;
+  int conv;      /* 1: short convolution + SiLU on q, k, v; 0: none */
+  int out_gate;  /* 1: gated RMSNorm of o with the g projection; 0: none */
 } gdn_layer_cfg_t;
 
 typedef struct {
@@ -325,19 +398,27 @@ typedef struct {
                             NVFP4 codes and scales itself (in its epilogue when
                             the tensor-core scan runs) and no quantizer pass
                             runs; the decode scale is 1 / o_g_enc. */
+  const float* x_g_enc;  /* NULL: x is quantized with its own amax (dynamic:
+                            an amax pass, then the quantizer).  Else a device
+                            FP32 encode scale for x (static, calibrated): one
+                            quantizer pass; the decode scale is 1 / x_g_enc. */
+  const float* conv_w;   /* cfg->conv: FP32 [2*H*dk + H*dv, 4] */
+  const float* g_g;      /* cfg->out_gate: decode scale of the g rows */
+  const float* norm_w;   /* cfg->out_gate: RMSNorm weight FP32 [dv] */
 } gdn_layer_weights_t;
 
 enum {
   GDN_WS_X_CODES = 0, GDN_WS_X_SCALES, GDN_WS_X_G, GDN_WS_QKV, GDN_WS_LOG_ALPHA,
   GDN_WS_BETA, GDN_WS_O, GDN_WS_O_CODES, GDN_WS_O_SCALES, GDN_WS_O_G,
-  GDN_WS_QUANT, GDN_WS_SCAN, GDN_WS_COUNT
+  GDN_WS_QUANT, GDN_WS_SCAN, GDN_WS_QKV_CONV, GDN_WS_G, GDN_WS_O_GATED, GDN_WS_COUNT
 };
 
 size_t gdn_layer_workspace_size(const gdn_layer_cfg_t* cfg);
 /* offsets[GDN_WS_COUNT] in bytes from ws: x codes, x scales (TILED), x decode
  * scale, qkv bf16 [B*T, 2*H*dk + H*dv], log_alpha / beta FP32 [B*T, H],
  * o bf16 [B*T, H*dv], o codes / scales / decode scale, quantizer and scan
- * scratch. */
+ * scratch, and (empty unless cfg->conv / cfg->out_gate) the convolved qkv,
+ * g bf16 [B*T, H*dv] and the gated o bf16 [B*T, H*dv]. */
 int gdn_layer_workspace_offsets(const gdn_layer_cfg_t* cfg, int64_t* offsets);
 
 int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg,

@@ -23,7 +23,7 @@ EPI_STORE_BF16, EPI_STORE_F32, EPI_LOG_ALPHA, EPI_BETA = 0, 1, 2, 3
 MAX_SEGMENTS = 8
 DR_L2NORM_QK, DR_O_FP32, DR_MMA_SYNC, DR_DECAYED_READ = 1, 2, 4, 8
 (WS_X_CODES, WS_X_SCALES, WS_X_G, WS_QKV, WS_LOG_ALPHA, WS_BETA, WS_O, WS_O_CODES,
- WS_O_SCALES, WS_O_G, WS_QUANT, WS_SCAN, WS_COUNT) = range(13)
+ WS_O_SCALES, WS_O_G, WS_QUANT, WS_SCAN, WS_QKV_CONV, WS_G, WS_O_GATED, WS_COUNT) = range(16)
 
 c_i64 = ctypes.c_int64
 c_vp = ctypes.c_void_p
@@ -44,13 +44,13 @@ class Segment(ctypes.Structure):
 
 class LayerCfg(ctypes.Structure):
     _fields_ = [("B", c_i64), ("T", c_i64), ("d_model", c_i64), ("H", ctypes.c_int),
-                ("dk", ctypes.c_int), ("dv", ctypes.c_int)]
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("conv", ctypes.c_int), ("out_gate", ctypes.c_int)]
 
 
 class LayerWeights(ctypes.Structure):
     _fields_ = [("w_qkvab", Nvfp4), ("g_q", c_vp), ("g_k", c_vp), ("g_v", c_vp), ("g_a", c_vp),
                 ("g_b", c_vp), ("w_out", Nvfp4), ("g_out", c_vp), ("A_log", c_vp), ("dt_bias", c_vp),
-                ("o_g_enc", c_vp)]
+                ("o_g_enc", c_vp), ("x_g_enc", c_vp), ("conv_w", c_vp), ("g_g", c_vp), ("norm_w", c_vp)]
 
 
 _LIB = None
@@ -69,14 +69,20 @@ def lib():
             "gdn_version": (ctypes.c_char_p, []),
             "gdn_stream_check": (ctypes.c_int, [c_vp]),
             "gdn_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, c_vp]),
+            "gdn_fp4_mma_ceiling": (ctypes.c_int, [c_i64, ctypes.POINTER(ctypes.c_int), c_vp]),
             "gdn_quantize_workspace_size": (ctypes.c_size_t, []),
             "gdn_scales_tiled_bytes": (ctypes.c_size_t, [c_i64, c_i64]),
             "gdn_quantize_nvfp4": (ctypes.c_int, [c_vp, ctypes.c_int, c_i64, c_i64, c_i64, ctypes.c_int, c_vp,
                                                   c_vp, c_vp, ctypes.c_int, c_i64, c_vp, c_vp, ctypes.c_size_t,
                                                   c_vp]),
+            "gdn_amax_update": (ctypes.c_int, [c_vp, ctypes.c_int, c_i64, c_i64, c_i64, c_vp, c_vp]),
+            "gdn_encode_scale_from_amax": (ctypes.c_int, [c_vp, c_vp, c_vp]),
             "gdn_gemm_nvfp4": (ctypes.c_int, [ctypes.POINTER(Nvfp4), c_vp, ctypes.POINTER(Nvfp4), c_i64, c_i64,
                                               c_i64, ctypes.POINTER(Segment), ctypes.c_int, c_vp]),
             "gdn_gates": (ctypes.c_int, [c_vp, c_vp, c_i64, ctypes.c_int, c_vp, c_vp, c_vp, c_vp, c_vp]),
+            "gdn_short_conv": (ctypes.c_int, [c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp]),
+            "gdn_gated_rmsnorm": (ctypes.c_int, [c_vp, c_vp, c_i64, ctypes.c_int, ctypes.c_int, c_vp, c_vp, c_vp,
+                                                 c_vp]),
             "gdn_delta_rule_workspace_size": (ctypes.c_size_t, [c_i64, c_i64, ctypes.c_int, ctypes.c_int,
                                                                 ctypes.c_int]),
             "gdn_delta_rule_fwd": (ctypes.c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_vp, c_i64,
@@ -101,8 +107,10 @@ def lib():
 
 
 EXPORTED = ("gdn_status_string", "gdn_last_error", "gdn_version", "gdn_stream_check", "gdn_selftest_bounded_wait",
-            "gdn_quantize_workspace_size", "gdn_scales_tiled_bytes", "gdn_quantize_nvfp4", "gdn_gemm_nvfp4",
-            "gdn_gates", "gdn_delta_rule_workspace_size", "gdn_delta_rule_fwd", "gdn_delta_rule_step",
+            "gdn_fp4_mma_ceiling",
+            "gdn_quantize_workspace_size", "gdn_scales_tiled_bytes", "gdn_quantize_nvfp4", "gdn_amax_update",
+            "gdn_encode_scale_from_amax", "gdn_gemm_nvfp4",
+            "gdn_gates", "gdn_short_conv", "gdn_gated_rmsnorm", "gdn_delta_rule_workspace_size", "gdn_delta_rule_fwd", "gdn_delta_rule_step",
             "gdn_layer_workspace_size",
             "gdn_layer_workspace_offsets", "gdn_layer_fwd", "gdn_layer_fwd_static_ws")
 LAYER_STATIC_WS_BYTES = 32 << 20
@@ -119,6 +127,12 @@ def check(status):
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _row_stride(x):
+    """Elements between the rows of a 2-D tensor (its width when empty, whose
+    strides torch leaves arbitrary)."""
+    return x.stride(0) if x.numel() else x.shape[1]
 
 
 def _stream(stream=None):
@@ -142,6 +156,14 @@ def stream_check(stream=None):
     check(lib().gdn_stream_check(_stream(stream)))
 
 
+def fp4_mma_ceiling(iters, stream=None):
+    """Enqueue the FP4 MMA ceiling kernel (one CTA per SM, iters x 4 MMAs of
+    128 x 256 x 64 each); returns the FLOPs it performs."""
+    ctas = ctypes.c_int(0)
+    check(lib().gdn_fp4_mma_ceiling(iters, ctypes.byref(ctas), _stream(stream)))
+    return 2.0 * 128 * 256 * 64 * 4 * iters * ctas.value
+
+
 # -------------------------------------------------------------- quantizer --
 def scales_tiled_bytes(rows, cols):
     return int(lib().gdn_scales_tiled_bytes(rows, cols))
@@ -158,7 +180,7 @@ def gdn_quantize_nvfp4(x, g_enc=None, layout="tiled", codes=None, scales=None, s
     filled from row ``sf_row_offset`` on."""
     if x.dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("x must be bf16 or float32")
-    if not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+    if not x.is_cuda or x.dim() != 2 or (x.numel() and x.stride(1) != 1):
         raise ValueError("x must be a 2-D CUDA tensor with unit column stride")
     rows, cols = x.shape
     dev = x.device
@@ -187,10 +209,63 @@ def gdn_quantize_nvfp4(x, g_enc=None, layout="tiled", codes=None, scales=None, s
     if ws is None and mode == QUANT_DYNAMIC:
         ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
     check(L.gdn_quantize_nvfp4(_ptr(x), DTYPE_F32 if x.dtype == torch.float32 else DTYPE_BF16, rows, cols,
-                               x.stride(0), mode, _ptr(g_enc), _ptr(codes), _ptr(scales),
+                               _row_stride(x), mode, _ptr(g_enc), _ptr(codes), _ptr(scales),
                                SF_TILED if tiled else SF_LINEAR, sf_row_offset, _ptr(g_out), _ptr(ws),
                                wsz if ws is not None else 0, _stream(stream)))
     return codes, scales, g_out
+
+
+# ------------------------------------------------------------ calibration --
+def gdn_amax_update(x, amax, stream=None):
+    """Fold max |x| of a 2-D bf16 / FP32 CUDA tensor (unit column stride) into
+    ``amax``, a 1-element FP32 CUDA tensor holding a running maximum."""
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("x must be bf16 or float32")
+    if not x.is_cuda or x.dim() != 2 or (x.numel() and x.stride(1) != 1):
+        raise ValueError("x must be a 2-D CUDA tensor with unit column stride")
+    _need(amax, torch.float32, "amax", x.device)
+    rows, cols = x.shape
+    check(lib().gdn_amax_update(_ptr(x), DTYPE_F32 if x.dtype == torch.float32 else DTYPE_BF16, rows, cols,
+                                _row_stride(x), _ptr(amax), _stream(stream)))
+    return amax
+
+
+def gdn_encode_scale_from_amax(amax, g_enc=None, stream=None):
+    """The encode scale 2688 / amax of a calibrated amax (1-element FP32 CUDA
+    tensors)."""
+    _need(amax, torch.float32, "amax")
+    if g_enc is None:
+        g_enc = torch.empty(1, dtype=torch.float32, device=amax.device)
+    _need(g_enc, torch.float32, "g_enc", amax.device)
+    check(lib().gdn_encode_scale_from_amax(_ptr(amax), _ptr(g_enc), _stream(stream)))
+    return g_enc
+
+
+def calibrate_layer(weights, batches, stream=None):
+    """Static activation scales of the layer's two quantized inputs, each
+    calibrated on its own: x (the input of the q/k/v/a/b projection) and o
+    (the input of the output projection).  ``batches``: bf16 CUDA tensors
+    [B, T, d_model].  Every batch's x folds into x's running amax; the layer
+    runs on it with dynamic scales and its o folds into o's.  Returns
+    (x_g_enc, o_g_enc), 1-element FP32 CUDA tensors for
+    ``weights.x_g_enc`` / ``weights.o_g_enc``."""
+    saved = (weights.x_g_enc, weights.o_g_enc)
+    weights.x_g_enc = weights.o_g_enc = None
+    try:
+        dev = batches[0].device
+        x_amax = torch.zeros(1, dtype=torch.float32, device=dev)
+        o_amax = torch.zeros(1, dtype=torch.float32, device=dev)
+        for x in batches:
+            B, T, D = x.shape
+            gdn_amax_update(x.view(B * T, D), x_amax, stream=stream)
+            _, _, ws = gdn_layer_fwd(weights, x, want_state=False, stream=stream)
+            off = gdn_layer_workspace_offsets(weights.cfg(B, T))
+            HV = weights.H * weights.dv
+            o = ws[off[WS_O]:off[WS_O] + B * T * HV * 2].view(torch.bfloat16).view(B * T, HV)
+            gdn_amax_update(o, o_amax, stream=stream)
+        return gdn_encode_scale_from_amax(x_amax, stream=stream), gdn_encode_scale_from_amax(o_amax, stream=stream)
+    finally:
+        weights.x_g_enc, weights.o_g_enc = saved
 
 
 # ------------------------------------------------------------------- GEMM --
@@ -256,6 +331,50 @@ def gdn_gates(a, b, A_log, dt_bias, log_alpha=None, beta=None, stream=None):
     return log_alpha, beta
 
 
+# ------------------------------------------------- convolution and norm --
+def gdn_short_conv(x, w, state_in=None, y=None, state_out=None, stream=None):
+    """Causal depthwise convolution of width 4 + SiLU over the channels of x
+    (bf16 [B, T, C], unit channel stride); w FP32 [C, 4]; state_in / state_out
+    bf16 [B, 3, C] or None.  Returns y (bf16 [B, T, C])."""
+    _need(x, torch.bfloat16, "x")
+    _need(w, torch.float32, "w")
+    if x.dim() != 3 or (x.numel() and x.stride(2) != 1):
+        raise ValueError("x must be [B, T, C] with unit channel stride")
+    B, T, C = x.shape
+    if T > 1 and B > 1 and x.stride(0) != T * x.stride(1):
+        raise ValueError("x: batch stride must be T * token stride")
+    ld_x = x.stride(1) if T > 1 else (x.stride(0) if B > 1 else C)
+    if y is None:
+        y = torch.empty((B, T, C), dtype=torch.bfloat16, device=x.device)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        if t is not None:
+            _need(t, torch.bfloat16, n)
+            if not t.is_contiguous() or t.shape != (B, 3, C):
+                raise ValueError(f"{n} must be a contiguous [B, 3, C] tensor")
+    check(lib().gdn_short_conv(_ptr(x), B, T, C, ld_x, _ptr(w), _ptr(state_in), _ptr(y), C, _ptr(state_out),
+                               _stream(stream)))
+    return y
+
+
+def gdn_gated_rmsnorm(o, g, gamma, H, y=None, amax=None, stream=None):
+    """o, g bf16 [M, H*dv] contiguous; gamma FP32 [dv].  Returns
+    y = o / sqrt(mean_dv(o^2) + 1e-6) * gamma * SiLU(g) per (token, head), bf16;
+    folds max |y| into ``amax`` (1-element FP32) when given."""
+    _need(o, torch.bfloat16, "o")
+    _need(g, torch.bfloat16, "g")
+    _need(gamma, torch.float32, "gamma")
+    if not (o.is_contiguous() and g.is_contiguous()) or o.shape != g.shape or o.dim() != 2:
+        raise ValueError("o, g must be contiguous [M, H*dv]")
+    M, HV = o.shape
+    if y is None:
+        y = torch.empty_like(o)
+    if amax is not None:
+        _need(amax, torch.float32, "amax")
+    check(lib().gdn_gated_rmsnorm(_ptr(o), _ptr(g), M, H, HV // H, _ptr(gamma), _ptr(y), _ptr(amax),
+                                  _stream(stream)))
+    return y
+
+
 # ------------------------------------------------------------- delta rule --
 def _token_stride(t, name):
     """Elements between consecutive tokens of a [B, T, H, d] tensor whose
@@ -274,11 +393,13 @@ def _token_stride(t, name):
 
 
 def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=False, o=None, S_T=None,
-                       want_state=True, stream=None, mma_sync=False):
+                       want_state=True, stream=None, mma_sync=False, use_workspace=True):
     """q, k [B, T, H, dk], v [B, T, H, dv] bf16 (heads contiguous, token stride
     free); log_alpha, beta FP32 [B, T, H] contiguous; S0 FP32 [B, H, dk, dv].
     ``mma_sync`` selects the warp-level mma.sync kernel where the tcgen05 one
-    would run.  Returns (o [B, T, H, dv] bf16 or FP32, S_T FP32 or None)."""
+    would run; ``use_workspace=False`` passes no workspace (long sequences on
+    few chains then run in one piece instead of segments).
+    Returns (o [B, T, H, dv] bf16 or FP32, S_T FP32 or None)."""
     lds = []
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
@@ -302,7 +423,7 @@ def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=Fa
             raise ValueError("S0 must be contiguous")
     flags = (DR_L2NORM_QK if l2norm else 0) | (DR_O_FP32 if o_fp32 else 0) | (DR_MMA_SYNC if mma_sync else 0)
     L = lib()
-    wsz = int(L.gdn_delta_rule_workspace_size(B, T, H, dk, dv))
+    wsz = int(L.gdn_delta_rule_workspace_size(B, T, H, dk, dv)) if use_workspace else 0
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev) if wsz else None
     check(L.gdn_delta_rule_fwd(_ptr(q), _ptr(k), _ptr(v), lds[0], lds[1], lds[2], _ptr(log_alpha),
                                _ptr(beta), _ptr(S0), B, T, H, dk, dv, flags, _ptr(o), _ptr(S_T), _ptr(ws), wsz,
@@ -349,20 +470,28 @@ def gdn_delta_rule_step(q, k, v, log_alpha, beta, S=None, l2norm=True, o_fp32=Fa
 class QuantizedLayerWeights:
     """NVFP4 weights of one layer, quantized on the device by the library:
     q, k, v, a, b share one [2*H*dk + H*dv + 2*H, d_model] operand (each with
-    its own decode scale), out is [d_model, H*dv].  ``o_g_enc`` (a 1-element
-    FP32 CUDA tensor, default None) is a static encode scale for the output
-    projection's activation; None quantizes o with its own amax."""
+    its own decode scale), out is [d_model, H*dv].  ``x_g_enc`` and
+    ``o_g_enc`` (1-element FP32 CUDA tensors, default None) are static encode
+    scales for the two quantized activations, x and o (``calibrate_layer``);
+    None quantizes that activation with its own amax."""
 
-    def __init__(self, W, A_log, dt_bias, H, dk, dv, device="cuda", stream=None):
+    def __init__(self, W, A_log, dt_bias, H, dk, dv, device="cuda", stream=None, conv_w=None, norm_w=None):
         d_model = W["q"].shape[1]
         self.H, self.dk, self.dv, self.d_model = H, dk, dv, d_model
+        names = ["q", "k", "v", "a", "b"]
         rows = [H * dk, H * dk, H * dv, H, H]
+        self.out_gate = 1 if "g" in W else 0
+        if self.out_gate:
+            if norm_w is None:
+                raise ValueError("the output gate needs norm_w")
+            names.append("g")
+            rows.append(H * dv)
         n_total = sum(rows)
         self.codes = torch.empty((n_total, d_model // 2), dtype=torch.uint8, device=device)
         self.scales = torch.zeros(scales_tiled_bytes(n_total, d_model), dtype=torch.uint8, device=device)
         self.g = {}
         r0 = 0
-        for name, nr in zip(("q", "k", "v", "a", "b"), rows):
+        for name, nr in zip(names, rows):
             w = torch.as_tensor(W[name], dtype=torch.float32).to(device).contiguous()
             _, _, g = gdn_quantize_nvfp4(w, codes=self.codes[r0:r0 + nr], scales=self.scales, sf_row_offset=r0,
                                          stream=stream)
@@ -373,6 +502,13 @@ class QuantizedLayerWeights:
         self.A_log = torch.as_tensor(A_log, dtype=torch.float32).to(device).contiguous()
         self.dt_bias = torch.as_tensor(dt_bias, dtype=torch.float32).to(device).contiguous()
         self.o_g_enc = None
+        self.x_g_enc = None
+        self.conv = 0 if conv_w is None else 1
+        self.conv_w = None if conv_w is None else torch.as_tensor(conv_w, dtype=torch.float32).to(device).contiguous()
+        self.norm_w = None if norm_w is None else torch.as_tensor(norm_w, dtype=torch.float32).to(device).contiguous()
+
+    def cfg(self, B, T):
+        return layer_cfg(B, T, self.d_model, self.H, self.dk, self.dv, self.conv, self.out_gate)
 
     def struct(self):
         s = LayerWeights()
@@ -385,11 +521,19 @@ class QuantizedLayerWeights:
         if self.o_g_enc is not None:
             _need(self.o_g_enc, torch.float32, "o_g_enc")
             s.o_g_enc = self.o_g_enc.data_ptr()
+        if self.x_g_enc is not None:
+            _need(self.x_g_enc, torch.float32, "x_g_enc")
+            s.x_g_enc = self.x_g_enc.data_ptr()
+        if self.conv_w is not None:
+            s.conv_w = self.conv_w.data_ptr()
+        if self.out_gate:
+            s.g_g = self.g["g"].data_ptr()
+            s.norm_w = self.norm_w.data_ptr()
         return s
 
 
-def layer_cfg(B, T, d_model, H, dk, dv):
-    return LayerCfg(B, T, d_model, H, dk, dv)
+def layer_cfg(B, T, d_model, H, dk, dv, conv=0, out_gate=0):
+    return LayerCfg(B, T, d_model, H, dk, dv, conv, out_gate)
 
 
 def gdn_layer_workspace_size(cfg):
@@ -408,7 +552,7 @@ def gdn_layer_fwd(weights, x, S0=None, want_state=True, y=None, S_T=None, ws=Non
     if not x.is_contiguous() or x.dim() != 3:
         raise ValueError("x must be a contiguous [B, T, d_model] tensor")
     B, T, D = x.shape
-    cfg = layer_cfg(B, T, D, weights.H, weights.dk, weights.dv)
+    cfg = weights.cfg(B, T)
     dev = x.device
     if y is None:
         y = torch.empty_like(x)
@@ -432,7 +576,7 @@ def gdn_layer_fwd_static_ws(weights, x, S0=None, want_state=True, y=None, S_T=No
     if not x.is_contiguous() or x.dim() != 3:
         raise ValueError("x must be a contiguous [B, T, d_model] tensor")
     B, T, D = x.shape
-    cfg = layer_cfg(B, T, D, weights.H, weights.dk, weights.dv)
+    cfg = weights.cfg(B, T)
     if y is None:
         y = torch.empty_like(x)
     if S_T is None and want_state:

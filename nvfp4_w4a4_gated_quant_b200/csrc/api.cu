@@ -167,6 +167,12 @@ int gdn_stream_check(gdn_stream_t stream) {
   return word;
 }
 
+int gdn_fp4_mma_ceiling(int64_t iters, int* ctas, gdn_stream_t stream) {
+  if (iters <= 0 || iters > ((int64_t)1 << 32) || !ctas) return GDN_ERR_INVALID_ARG;
+  *ctas = num_sms();
+  return launch_fp4_mma_ceiling(iters, *ctas, as_stream(stream));
+}
+
 int gdn_selftest_bounded_wait(uint32_t poll_limit, gdn_stream_t stream) {
   if (poll_limit == 0 || poll_limit > (1u << 26)) return GDN_ERR_INVALID_ARG;
   int* status = device_status_word();
@@ -191,6 +197,49 @@ int gdn_quantize_nvfp4(const void* x, int x_dtype, int64_t rows, int64_t cols, i
   return launch_quantize(x, x_dtype, rows, cols, ld_x, mode, g_enc_in, codes, scales,
                          sf_layout == GDN_SF_TILED ? 1 : 0, sf_row_offset, g_out, static_cast<unsigned*>(ws),
                          as_stream(stream));
+}
+
+int gdn_amax_update(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x, float* amax,
+                    gdn_stream_t stream) {
+  if (rows < 0 || cols <= 0 || ld_x < cols || !amax) return GDN_ERR_INVALID_ARG;
+  if (x_dtype != GDN_DTYPE_BF16 && x_dtype != GDN_DTYPE_F32) return GDN_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return GDN_ERR_UNSUPPORTED_SHAPE;
+  const int64_t per16 = x_dtype == GDN_DTYPE_F32 ? 4 : 8;
+  if (rows > 0 && (!x || !aligned(x, 16) || ld_x % per16 != 0)) return x ? GDN_ERR_ALIGNMENT : GDN_ERR_INVALID_ARG;
+  if (!aligned(amax, 4)) return GDN_ERR_ALIGNMENT;
+  return launch_amax_update(x, x_dtype, rows, cols, ld_x, amax, as_stream(stream));
+}
+
+int gdn_encode_scale_from_amax(const float* amax, float* g_enc, gdn_stream_t stream) {
+  if (!amax || !g_enc) return GDN_ERR_INVALID_ARG;
+  if (!aligned(amax, 4) || !aligned(g_enc, 4)) return GDN_ERR_ALIGNMENT;
+  return launch_encode_scale(amax, g_enc, as_stream(stream));
+}
+
+int gdn_short_conv(const void* x, int64_t B, int64_t T, int64_t C, int64_t ld_x, const float* w, const void* state_in,
+                   void* y, int64_t ld_y, void* state_out, gdn_stream_t stream) {
+  if (B < 0 || T < 0 || C <= 0 || ld_x < C || ld_y < C || !w) return GDN_ERR_INVALID_ARG;
+  if (C % 8 != 0 || B > 65535 || T > (int64_t)65535 * 64) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (B > 0 && T > 0) {
+    if (!x || !y) return GDN_ERR_INVALID_ARG;
+    if (x == y) return GDN_ERR_INVALID_ARG;   // the window reads earlier inputs: no in-place call
+    if (!aligned(x, 16) || !aligned(y, 16) || ld_x % 8 || ld_y % 8) return GDN_ERR_ALIGNMENT;
+  }
+  if (!aligned(w, 16) || (state_in && !aligned(state_in, 16)) || (state_out && !aligned(state_out, 16)))
+    return GDN_ERR_ALIGNMENT;
+  return launch_short_conv(static_cast<const uint16_t*>(x), B, T, C, ld_x, w, static_cast<const uint16_t*>(state_in),
+                           static_cast<uint16_t*>(y), ld_y, static_cast<uint16_t*>(state_out), as_stream(stream));
+}
+
+int gdn_gated_rmsnorm(const void* o, const void* g, int64_t M, int H, int dv, const float* gamma, void* y,
+                      float* amax, gdn_stream_t stream) {
+  if (M < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+  if (dv != 32 && dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED_SHAPE;
+  if (M > 0 && (!o || !g || !gamma || !y)) return GDN_ERR_INVALID_ARG;
+  if ((o && !aligned(o, 2)) || (g && !aligned(g, 2)) || (y && !aligned(y, 2)) || (amax && !aligned(amax, 4)))
+    return GDN_ERR_ALIGNMENT;
+  return launch_gated_rmsnorm(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(g), M, H, dv, gamma,
+                              static_cast<uint16_t*>(y), amax, as_stream(stream));
 }
 
 int gdn_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B, int64_t M, int64_t N, int64_t K,
@@ -227,19 +276,13 @@ int gdn_gates(const float* a, const float* b, int64_t M, int H, const float* A_l
 }
 
 size_t gdn_delta_rule_workspace_size(int64_t B, int64_t T, int H, int dk, int dv) {
-  (void)B;
-  (void)T;
-  (void)H;
-  (void)dk;
-  (void)dv;
-  return 0;
+  if (B <= 0 || T <= 0 || H <= 0) return 0;
+  return delta_rule_tc_workspace(B, T, H, dk, dv);
 }
 
 int gdn_delta_rule_fwd(const void* q, const void* k, const void* v, int64_t ld_q, int64_t ld_k, int64_t ld_v,
                        const float* log_alpha, const float* beta, const float* S0, int64_t B, int64_t T, int H, int dk,
                        int dv, int flags, void* o, float* S_T, void* ws, size_t ws_bytes, gdn_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (B < 0 || T < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
   if (flags & ~(GDN_DR_L2NORM_QK | GDN_DR_O_FP32 | GDN_DR_MMA_SYNC)) return GDN_ERR_INVALID_ARG;
   if ((dk != 32 && dk != 64 && dk != 128) || (dv != 32 && dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED_SHAPE;
@@ -253,9 +296,10 @@ int gdn_delta_rule_fwd(const void* q, const void* k, const void* v, int64_t ld_q
       return GDN_ERR_ALIGNMENT;
   }
   if ((S0 && !aligned(S0, 4)) || (S_T && !aligned(S_T, 4))) return GDN_ERR_ALIGNMENT;
+  if (ws && !aligned(ws, 256)) return GDN_ERR_ALIGNMENT;
   return launch_delta_rule(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
                            static_cast<const uint16_t*>(v), ld_q, ld_k, ld_v, log_alpha, beta, S0, B, T, H, dk, dv,
-                           flags, o, S_T, nullptr, as_stream(stream));
+                           flags, o, S_T, nullptr, as_stream(stream), nullptr, ws, ws ? ws_bytes : 0);
 }
 
 int gdn_delta_rule_step(const void* q, const void* k, const void* v, int64_t ld_q, int64_t ld_k, int64_t ld_v,

@@ -763,14 +763,14 @@ int launch_dk(const Args& a, int dvs, int64_t chains, cudaStream_t stream) {
 int launch_delta_rule(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                       int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
                       int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
-                      cudaStream_t stream, const OQuant* oq) {
+                      cudaStream_t stream, const OQuant* oq, void* ws, size_t ws_bytes) {
   const int64_t chains = B * H;
   if (chains == 0) return GDN_OK;
   if (oq && (flags & GDN_DR_O_FP32)) return GDN_ERR_UNSUPPORTED_SHAPE;   // o is quantized from its bf16 values
   // the tensor-core kernel stores o and S_T in 16-byte vectors
   if (!(flags & GDN_DR_MMA_SYNC) && delta_rule_tc_supported(dk, dv, T) && aligned(o, 16) && (!S_T || aligned(S_T, 16)))
     return launch_delta_rule_tc(q, k, v, ld_q, ld_k, ld_v, log_alpha, beta, S0, B, T, H, dk, dv, flags, o, S_T,
-                                o_amax, stream, oq);
+                                o_amax, stream, oq, ws, ws_bytes);
   if (oq) {
     int st = launch_delta_rule(q, k, v, ld_q, ld_k, ld_v, log_alpha, beta, S0, B, T, H, dk, dv, flags, o, S_T, o_amax,
                                stream, nullptr);

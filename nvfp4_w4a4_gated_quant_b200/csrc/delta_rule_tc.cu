@@ -177,7 +177,21 @@ struct Args {
   int64_t T;
   int H, dv, nsplit;
   int l2norm;
-  void* o;
+  // segments: every sequence is cut into nseg pieces of T_seg tokens (the
+  // last one shorter), one CTA per (batch, segment, head, d_v slice); S0 and
+  // S_T are per (batch, segment, head) unless st_last_only, when S_T is the
+  // last segment's final state per (batch, head).  nseg = 1, T_seg = T: one
+  // piece per sequence.
+  int nseg;
+  int64_t T_seg;
+  int st_last_only;
+  // state columns per row of S0 / S_T (dv, or more when some slices carry
+  // other columns), and the number of leading slices whose v is taken as
+  // zero and whose initial state is the identity (they propagate the
+  // segment's state-transition matrix instead of its state)
+  int dv_state;
+  int zero_splits;
+  void* o;              // may be null: no o (nor its amax or NVFP4 codes)
   float* S_T;
   unsigned* o_amax;
   int* status;
@@ -192,13 +206,13 @@ struct Maps {
 };
 
 // The raw gates of chunk t0 (warp 7: two tokens per lane; zero past the end
-// of the sequence), fetched well before they are needed.
-__device__ __forceinline__ void fetch_gates(const Args& a, int64_t tok0, int h, int64_t t0, int lane, float (&la)[2],
-                                            float (&bs)[2]) {
+// of the segment, `len` tokens), fetched well before they are needed.
+__device__ __forceinline__ void fetch_gates(const Args& a, int64_t tok0, int h, int64_t t0, int64_t len, int lane,
+                                            float (&la)[2], float (&bs)[2]) {
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int64_t t = t0 + 2 * lane + e;
-    const bool ok = t < a.T;
+    const bool ok = t < len;
     la[e] = ok ? __ldg(a.log_alpha + (tok0 + t) * a.H + h) : 0.0f;
     bs[e] = ok ? __ldg(a.beta + (tok0 + t) * a.H + h) : 0.0f;
   }
@@ -440,13 +454,18 @@ __global__ void __launch_bounds__(NTP, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int chain = blockIdx.x / a.nsplit;
+  const int chain = blockIdx.x / a.nsplit;   // (batch, segment, head)
   const int split = blockIdx.x % a.nsplit;
-  const int b = chain / a.H, h = chain % a.H;
-  const int dv_off = split * DVS;
+  const int h = chain % a.H;
+  const int b = (chain / a.H) / a.nseg, p = (chain / a.H) % a.nseg;
+  const bool zero_v = split < a.zero_splits;
+  const int dv_off = zero_v ? 0 : (split - a.zero_splits) * DVS;     // the v / o columns of this slice
+  const int st_off = split * DVS;                                    // its S0 / S_T columns
   const int64_t T = a.T;
-  const int64_t tok0 = (int64_t)b * T;
-  const int64_t nchunks = (T + C - 1) / C;
+  const int64_t seg0 = (int64_t)p * a.T_seg;                         // the segment's first token
+  const int64_t len = T - seg0 < a.T_seg ? T - seg0 : a.T_seg;
+  const int64_t tok0 = (int64_t)b * T + seg0;
+  const int64_t nchunks = (len + C - 1) / C;
   constexpr int LD_ISSUER = NTP - 32;   // warp 11, lane 0: issues every chunk load
   constexpr int BAR_PG = 1, BAR_SG = 2, BAR_INV = 3;
 
@@ -492,13 +511,13 @@ __global__ void __launch_bounds__(NTP, 1)
   int kq0 = 0, kq1 = 0, v0 = 0, v1 = 0;
   if (tid == LD_ISSUER) {
     if (nchunks > 0) {
-      pipe_load_kq<DVS>(sb, &bar_ld[0], maps, b, h, 0, 0);
-      pipe_load_v<DVS>(sb, &bar_ld[0], maps, a, b, h, dv_off, 0, 0);
+      pipe_load_kq<DVS>(sb, &bar_ld[0], maps, b, h, seg0, 0);
+      pipe_load_v<DVS>(sb, &bar_ld[0], maps, a, b, h, dv_off, seg0, 0);
       kq0 = v0 = 1;
     }
     if (nchunks > 1) {
-      pipe_load_kq<DVS>(sb, &bar_ld[1], maps, b, h, C, 1);
-      pipe_load_v<DVS>(sb, &bar_ld[1], maps, a, b, h, dv_off, C, 1);
+      pipe_load_kq<DVS>(sb, &bar_ld[1], maps, b, h, seg0 + C, 1);
+      pipe_load_v<DVS>(sb, &bar_ld[1], maps, a, b, h, dv_off, seg0 + C, 1);
       kq1 = v1 = 1;
     }
   }
@@ -508,7 +527,7 @@ __global__ void __launch_bounds__(NTP, 1)
     // ======================================================== prep group
     const int colhalf = warp >> 2;
     float nla[2] = {0.f, 0.f}, nbs[2] = {0.f, 0.f};
-    if (warp == 7 && nchunks > 0) fetch_gates(a, tok0, h, 0, lane, nla, nbs);
+    if (warp == 7 && nchunks > 0) fetch_gates(a, tok0, h, 0, len, lane, nla, nbs);
     int64_t c = 0;
 #pragma unroll 1
     for (; c < nchunks; ++c) {
@@ -523,7 +542,7 @@ __global__ void __launch_bounds__(NTP, 1)
       // the gate factors of chunk c (raw gates fetched one chunk ahead)
       if (warp == 7) {
         const float la[2] = {nla[0], nla[1]}, bs[2] = {nbs[0], nbs[1]};
-        if (c + 1 < nchunks) fetch_gates(a, tok0, h, (c + 1) * C, lane, nla, nbs);
+        if (c + 1 < nchunks) fetch_gates(a, tok0, h, (c + 1) * C, len, lane, nla, nbs);
         fb[Fac::BE + 2 * lane] = bs[0];
         fb[Fac::BE + 2 * lane + 1] = bs[1];
         scan_gates(fb, la, bs, lane);
@@ -536,7 +555,7 @@ __global__ void __launch_bounds__(NTP, 1)
       // beta v in place
       for (int i = tid; i < C * DVS / 8; i += NPG) {
         const uint32_t off = (uint32_t)i * 16;
-        const float bt = be[(i >> 3) & 63];
+        const float bt = zero_v ? 0.0f : be[(i >> 3) & 63];
         float x[8];
         unpack_bf16x8(ld_s128(vb + off), x);
 #pragma unroll
@@ -783,7 +802,8 @@ __global__ void __launch_bounds__(NTP, 1)
         uint32_t v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          v[i] = __float_as_uint(a.S0 ? a.S0[((int64_t)chain * DK + r) * a.dv + dv_off + c0 + i] : 0.0f);
+          v[i] = __float_as_uint(zero_v ? (r == st_off + c0 + i ? 1.0f : 0.0f)
+                                 : a.S0 ? a.S0[((int64_t)chain * DK + r) * a.dv_state + st_off + c0 + i] : 0.0f);
         tmem_st_32x32b_x16(tmem + lane_off + PS + c0, v);
       }
       tc_wait_st();
@@ -797,7 +817,7 @@ __global__ void __launch_bounds__(NTP, 1)
       const int s = (int)(c & 1);
       const uint32_t ph = (uint32_t)(c >> 1) & 1u;
       const int64_t t0 = c * C;
-      const int valid = (int)(T - t0 < C ? T - t0 : C);
+      const int valid = (int)(len - t0 < C ? len - t0 : C);
       const uint32_t t3 = sb + M::t3(s), pb = sb + M::pt(s), vb = sb + M::vb(s);
       const float* fb = reinterpret_cast<const float*>(smem + M::F + (uint32_t)s * M::F_BYTES);
       tc_fence_before();
@@ -866,7 +886,7 @@ __global__ void __launch_bounds__(NTP, 1)
       tc_fence_after();
       // the [K; Q; W] tile of stage s is free: chunk c+2's k and q
       if (tid == LD_ISSUER && c + 2 < nchunks) {
-        pipe_load_kq<DVS>(sb, &bar_ld[s], maps, b, h, t0 + 2 * C, s);
+        pipe_load_kq<DVS>(sb, &bar_ld[s], maps, b, h, seg0 + t0 + 2 * C, s);
         if (s == 0) ++kq0; else ++kq1;
       }
       // ---- U = U~ - W S -> beta-V tile (quarters 2, 3: token rows in lanes 64..127)
@@ -912,11 +932,11 @@ __global__ void __launch_bounds__(NTP, 1)
       tc_fence_after();
       // the beta-V tile of stage s is free: chunk c+2's v
       if (tid == LD_ISSUER && c + 2 < nchunks) {
-        pipe_load_v<DVS>(sb, &bar_ld[s], maps, a, b, h, dv_off, t0 + 2 * C, s);
+        pipe_load_v<DVS>(sb, &bar_ld[s], maps, a, b, h, dv_off, seg0 + t0 + 2 * C, s);
         if (s == 0) ++v0; else ++v1;
       }
       // ---- o rows (quarters 0, 1: token rows in lanes 0..63), 32 columns at a time
-      if (quarter < 2) {
+      if (quarter < 2 && a.o) {
         const int t = quarter * 32 + lane;
         const int64_t row = tok0 + t0 + t;
 #pragma unroll 1
@@ -980,14 +1000,15 @@ __global__ void __launch_bounds__(NTP, 1)
       }
     }
     // the final state
-    if (c == nchunks && a.S_T && *abort_flag == 0) {
+    if (c == nchunks && a.S_T && *abort_flag == 0 && (!a.st_last_only || p == a.nseg - 1)) {
       const int r = quarter * 32 + lane;
+      const int64_t srow = a.st_last_only ? (int64_t)b * a.H + h : chain;
 #pragma unroll
       for (int n0 = 0; n0 < DVS; n0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lane_off + PS + n0, v);
         tc_wait_ld();
-        float4* dst = reinterpret_cast<float4*>(a.S_T + ((int64_t)chain * DK + r) * a.dv + dv_off + n0);
+        float4* dst = reinterpret_cast<float4*>(a.S_T + (srow * DK + r) * a.dv_state + st_off + n0);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)
           dst[cc] = make_float4(__uint_as_float(v[4 * cc]), __uint_as_float(v[4 * cc + 1]),
@@ -1014,8 +1035,9 @@ __global__ void __launch_bounds__(NTP, 1)
   // chunk loads still in flight after an early exit land before the CTA exits
   if (tid == LD_ISSUER) {
     // a stage whose k and q went out without its v: complete the phase
-    if (v0 < kq0) pipe_load_v<DVS>(sb, &bar_ld[0], maps, a, b, h, dv_off, (int64_t)(2 * (kq0 - 1)) * C, 0);
-    if (v1 < kq1) pipe_load_v<DVS>(sb, &bar_ld[1], maps, a, b, h, dv_off, (int64_t)(2 * (kq1 - 1) + 1) * C, 1);
+    if (v0 < kq0) pipe_load_v<DVS>(sb, &bar_ld[0], maps, a, b, h, dv_off, seg0 + (int64_t)(2 * (kq0 - 1)) * C, 0);
+    if (v1 < kq1)
+      pipe_load_v<DVS>(sb, &bar_ld[1], maps, a, b, h, dv_off, seg0 + (int64_t)(2 * (kq1 - 1) + 1) * C, 1);
     for (int k = consumed[0]; k < kq0; ++k) mbar_wait(&bar_ld[0], (uint32_t)k & 1u, a.status);
     for (int k = consumed[1]; k < kq1; ++k) mbar_wait(&bar_ld[1], (uint32_t)k & 1u, a.status);
   }
@@ -1043,31 +1065,138 @@ bool make_map_3d(CUtensorMap* map, const void* base, int64_t features, int64_t T
 }
 
 template <int DVS, bool O_F32>
-int launch_dvs(const Args& a, const Maps& m, int64_t chains, cudaStream_t stream) {
+int launch_dvs(const Args& a, const Maps& m, int64_t units, cudaStream_t stream) {
   const size_t smem = PMap<DVS>::BYTES + 1024;
   cudaError_t e =
       cudaFuncSetAttribute(delta_rule_pipe_kernel<DVS, O_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return record_cuda_error(e);
-  delta_rule_pipe_kernel<DVS, O_F32><<<(unsigned)(chains * a.nsplit), NTP, smem, stream>>>(a, m);
+  delta_rule_pipe_kernel<DVS, O_F32><<<(unsigned)(units * a.nsplit), NTP, smem, stream>>>(a, m);
   return check_launch();
 }
+
+int launch_args(const Args& a, const Maps& m, int64_t units, int dvs, bool f32, cudaStream_t stream) {
+  if (dvs == 128) return f32 ? launch_dvs<128, true>(a, m, units, stream) : launch_dvs<128, false>(a, m, units, stream);
+  return f32 ? launch_dvs<64, true>(a, m, units, stream) : launch_dvs<64, false>(a, m, units, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Segments: sequences cut into pieces that run in parallel.
+//
+// The chunk map of the recurrence is affine in the state: a segment takes its
+// entry state S to M S + B, where B is the segment's final state when it
+// starts from zero and M (d_k x d_k) is what the same steps do to the
+// identity with v taken as zero (the write term is the only one that does
+// not scale with S).  So with few (batch, head) chains and long sequences --
+// too few CTAs to cover the SMs, each walking a long chain of chunks -- the
+// sequence is cut into P segments:
+//   phase A  segments 0 .. P-2 run from [I | 0] (the identity block with
+//            v = 0, then the real v from a zero state): final [M_p | B_p];
+//   phase B  S_0 = S0, S_{p+1} = M_p S_p + B_p (FP32, P-1 small products);
+//   phase C  every segment runs again from its entry state S_p, writing o
+//            and, for the last one, S_T.
+// Phase A costs (d_k + d_v) / d_v times the state work of P-1 segments and
+// phase C one pass, but both run on P times as many CTAs.
+
+// E[b, p, h] = S_p for p = 0 .. nseg-1, S_0 = S0 (or 0), S_{p+1} = M_p S_p +
+// B_p with [M_p | B_p] = MB[b, p, h] ([d_k, d_k + dv]).  One CTA of 256
+// threads per (batch, head, 16 state columns): thread t owns row t/2 and
+// eight columns; the sixteen columns of S_p stay in shared memory.
+__global__ void __launch_bounds__(256) segment_combine_kernel(const float* __restrict__ MB,
+                                                              const float* __restrict__ S0, float* __restrict__ E,
+                                                              int H, int dv, int nseg) {
+  __shared__ float Ss[DK][16];
+  const int ncb = dv / 16;
+  const int cb = blockIdx.x % ncb, bh = blockIdx.x / ncb;
+  const int b = bh / H, h = bh % H;
+  const int tid = threadIdx.x, r = tid >> 1, c0 = (tid & 1) * 8;
+  const int col = cb * 16 + c0;
+  const int ld = DK + dv;
+  float st[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) st[e] = S0 ? S0[(((int64_t)b * H + h) * DK + r) * dv + col + e] : 0.0f;
+  for (int p = 0;; ++p) {
+    float* dst = E + ((((int64_t)b * nseg + p) * H + h) * DK + r) * dv + col;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[e] = st[e];
+    if (p + 1 == nseg) break;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) Ss[r][c0 + e] = st[e];
+    __syncthreads();
+    const float* mrow = MB + ((((int64_t)b * (nseg - 1) + p) * H + h) * DK + r) * ld;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = mrow[DK + col + e];
+#pragma unroll 4
+    for (int k = 0; k < DK; k += 4) {
+      const float4 m4 = *reinterpret_cast<const float4*>(mrow + k);
+      const float mk[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(mk[kk], Ss[k + kk][c0 + e], acc[e]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) st[e] = acc[e];
+  }
+}
+
+struct SegPlan {
+  int P = 1;
+  int64_t T_seg = 0;
+};
+
+// The segment count that minimises the chunk steps on the critical path --
+// waves of CTAs x (chunks per CTA + the pipeline's fill and drain, about four
+// chunk steps), plus one step per sequential product of phase B -- if it
+// beats one piece per sequence by a clear margin; d_v a multiple of 128 (the
+// identity block is one 128-column slice).
+SegPlan plan_segments(int64_t B, int64_t T, int H, int dv, int sms) {
+  SegPlan best;
+  if (dv % 128 != 0 || T <= 0 || B * H <= 0) return best;
+  constexpr int64_t kFill = 4;
+  const int64_t chains = B * H, nch = (T + C - 1) / C, sl = dv / 128;
+  int64_t plain_split = sl;
+  if (chains * sl * 2 <= sms) plain_split = 2 * sl;
+  double best_cost = 0.75 * (double)cdiv(chains * plain_split, sms) * (double)(nch + kFill);
+  for (int P = 2; P <= 64; ++P) {
+    const int64_t tc = cdiv(nch, P);
+    if ((P - 1) * tc >= nch) break;   // the last segment would be empty
+    const double cost =
+        (double)(cdiv(chains * (P - 1) * (1 + sl), sms) + cdiv(chains * P * sl, sms)) * (double)(tc + kFill) + (P - 1);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best.P = P;
+      best.T_seg = tc * C;
+    }
+  }
+  return best;
+}
+
+size_t seg_bytes_mb(int64_t B, int H, int dv, int P) { return (size_t)(B * (P - 1) * H) * DK * (DK + dv) * 4; }
+size_t seg_bytes_e(int64_t B, int H, int dv, int P) { return (size_t)(B * P * H) * DK * dv * 4; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
 bool delta_rule_tc_supported(int dk, int dv, int64_t T) { return dk == DK && dv % 64 == 0 && T < ((int64_t)1 << 31); }
 
+size_t delta_rule_tc_workspace(int64_t B, int64_t T, int H, int dk, int dv) {
+  if (!delta_rule_tc_supported(dk, dv, T)) return 0;
+  const SegPlan pl = plan_segments(B, T, H, dv, num_sms());
+  if (pl.P < 2) return 0;
+  return align256(seg_bytes_mb(B, H, dv, pl.P)) + seg_bytes_e(B, H, dv, pl.P);
+}
+
 int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
                          int64_t ld_v, const float* log_alpha, const float* beta, const float* S0, int64_t B,
                          int64_t T, int H, int dk, int dv, int flags, void* o, float* S_T, unsigned* o_amax,
-                         cudaStream_t stream, const OQuant* oq) {
+                         cudaStream_t stream, const OQuant* oq, void* ws, size_t ws_bytes) {
   const int64_t chains = B * H;
   if (chains == 0) return GDN_OK;
   if (!delta_rule_tc_supported(dk, dv, T)) return GDN_ERR_UNSUPPORTED_SHAPE;
   if (oq && (flags & GDN_DR_O_FP32)) return GDN_ERR_UNSUPPORTED_SHAPE;
-  // d_v slices of 128 columns unless the chains leave more than half the SMs idle
   const int sms = num_sms();
-  int dvs = (dv % 128 == 0) ? 128 : 64;
-  if (dvs == 128 && chains * (dv / 128) * 2 <= sms) dvs = 64;
   const bool f32 = (flags & GDN_DR_O_FP32) != 0;
   Maps m;
   memset(&m, 0, sizeof(m));
@@ -1082,8 +1211,12 @@ int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v
   a.T = T;
   a.H = H;
   a.dv = dv;
-  a.nsplit = dv / dvs;
   a.l2norm = (flags & GDN_DR_L2NORM_QK) ? 1 : 0;
+  a.nseg = 1;
+  a.T_seg = Tm;
+  a.st_last_only = 0;
+  a.dv_state = dv;
+  a.zero_splits = 0;
   a.o = o;
   a.S_T = S_T;
   a.o_amax = o_amax;
@@ -1094,8 +1227,45 @@ int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v
     a.oq_g_enc = oq->g_enc;
     a.oq_g_out = oq->g_out;
   }
-  if (dvs == 128) return f32 ? launch_dvs<128, true>(a, m, chains, stream) : launch_dvs<128, false>(a, m, chains, stream);
-  return f32 ? launch_dvs<64, true>(a, m, chains, stream) : launch_dvs<64, false>(a, m, chains, stream);
+  const SegPlan pl = plan_segments(B, T, H, dv, sms);
+  const size_t need = pl.P > 1 ? align256(seg_bytes_mb(B, H, dv, pl.P)) + seg_bytes_e(B, H, dv, pl.P) : 0;
+  if (pl.P > 1 && ws && ws_bytes >= need && aligned(ws, 256)) {
+    float* MB = static_cast<float*>(ws);
+    float* E = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(seg_bytes_mb(B, H, dv, pl.P)));
+    // phase A: segments 0 .. P-2 from [I | 0]; the state transition and the
+    // zero-start state of each, no o
+    Args pa = a;
+    pa.nseg = pl.P - 1;
+    pa.T_seg = pl.T_seg;
+    pa.S0 = nullptr;
+    pa.S_T = MB;
+    pa.dv_state = DK + dv;
+    pa.zero_splits = 1;
+    pa.nsplit = 1 + dv / 128;
+    pa.o = nullptr;
+    pa.o_amax = nullptr;
+    pa.oq_codes = nullptr;
+    int st = launch_args(pa, m, B * (pl.P - 1) * H, 128, f32, stream);
+    if (st) return st;
+    // phase B: the entry state of every segment
+    segment_combine_kernel<<<(unsigned)(B * H * (dv / 16)), 256, 0, stream>>>(MB, S0, E, H, dv, pl.P);
+    st = check_launch();
+    if (st) return st;
+    // phase C: every segment from its entry state
+    Args pc = a;
+    pc.nseg = pl.P;
+    pc.T_seg = pl.T_seg;
+    pc.S0 = E;
+    pc.st_last_only = 1;
+    pc.nsplit = dv / 128;
+    return launch_args(pc, m, B * pl.P * H, 128, f32, stream);
+  }
+  // one piece per sequence: d_v slices of 128 columns unless the chains leave
+  // more than half the SMs idle
+  int dvs = (dv % 128 == 0) ? 128 : 64;
+  if (dvs == 128 && chains * (dv / 128) * 2 <= sms) dvs = 64;
+  a.nsplit = dv / dvs;
+  return launch_args(a, m, chains, dvs, f32, stream);
 }
 
 }  // namespace gdn

@@ -556,7 +556,90 @@ bool make_out_map(CUtensorMap* map, const gdn_epilogue_segment_t& sg, int64_t M)
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The FP4 tensor-core ceiling of this GEMM's MMA: M = 128, N = 256, K = 64
+// kind::mxf4nvf4 with block-16 scales, issued back to back by one converged
+// warp from operand tiles resident in shared memory (E2M1 codes from a
+// hash, so the multipliers see ordinary data) and scales resident in TMEM --
+// no loads, no scale hand-off, no epilogue.  One CTA per SM; the GEMM's
+// achieved rate divided by this rate is its efficiency against what the
+// tensor pipe delivers at the clock and power of the moment.
+constexpr int CEIL_THREADS = 128;
+// more shared memory than two CTAs can hold on one SM: one CTA per SM (each
+// allocates all of TMEM)
+constexpr size_t CEIL_SMEM = 120 * 1024;
+static_assert(CEIL_SMEM >= 1024 + A_BYTES + B_BYTES + 64, "ceiling tiles");
+
+__global__ void __launch_bounds__(CEIL_THREADS, 1) fp4_mma_ceiling_kernel(int64_t iters, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sb - sraw);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + A_BYTES + B_BYTES);
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + A_BYTES + B_BYTES + 8);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // codes: any nibble is a valid E2M1 value
+  for (int i = tid; i < (A_BYTES + B_BYTES) / 4; i += CEIL_THREADS) {
+    uint32_t x = (uint32_t)i * 2654435761u + 0x9E3779B9u * (blockIdx.x + 1);
+    x ^= x >> 15;
+    x *= 0x2C1B3C6Du;
+    x ^= x >> 12;
+    reinterpret_cast<uint32_t*>(smem)[i] = x;
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_ptr, TMEM_COLS);
+    tmem_relinquish();
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  {
+    // every scale 1.0 (E4M3 0x38) in the 48 columns the MMAs read
+    uint32_t one[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) one[i] = 0x38383838u;
+    const uint32_t col = tmem + ((uint32_t)(warp * 32) << 16) + SF_COL;
+    tmem_st_32x32b_x16(col, one);
+    tmem_st_32x32b_x16(col + 16, one);
+    tmem_st_32x32b_x16(col + 32, one);
+    tc_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    const uint32_t a_s = sb, b_s = sb + A_BYTES;
+    const uint32_t acc = tmem + ACC_COL, sf = tmem + SF_COL;
+    for (int64_t it = 0; it < iters; ++it)
+#pragma unroll
+      for (int j = 0; j < BK / KSTEP; ++j)
+        tc_mma_nvf4_warp(acc, desc_sw128(a_s + j * 32), desc_sw128(b_s + j * 32), kIdesc, sf + j * 4,
+                         sf + SFB_OFF + j * SFB_PER_K, (it > 0 || j > 0) ? 1u : 0u);
+    tc_commit_warp(bar);
+    mbar_wait(bar, 0, status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
 }  // namespace
+
+int launch_fp4_mma_ceiling(int64_t iters, int ctas, cudaStream_t stream) {
+  cudaError_t e =
+      cudaFuncSetAttribute(fp4_mma_ceiling_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CEIL_SMEM);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  fp4_mma_ceiling_kernel<<<ctas, CEIL_THREADS, CEIL_SMEM, stream>>>(iters, device_status_word());
+  return check_launch();
+}
 
 int launch_gemm_nvfp4(const gdn_nvfp4_t* A, const float* g_a, const gdn_nvfp4_t* B, int64_t M, int64_t N, int64_t K,
                       const gdn_epilogue_segment_t* segs, int n_segs, cudaStream_t stream) {

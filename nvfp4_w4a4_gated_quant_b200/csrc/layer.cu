@@ -14,7 +14,8 @@ namespace {
 int64_t align256(int64_t x) { return (x + 255) & ~(int64_t)255; }
 
 bool cfg_ok(const gdn_layer_cfg_t* c) {
-  return c && c->B >= 0 && c->T >= 0 && c->d_model > 0 && c->H > 0 && c->dk > 0 && c->dv > 0;
+  return c && c->B >= 0 && c->T >= 0 && c->d_model > 0 && c->H > 0 && c->dk > 0 && c->dv > 0 &&
+         (c->conv == 0 || c->conv == 1) && (c->out_gate == 0 || c->out_gate == 1);
 }
 
 int layout(const gdn_layer_cfg_t* c, int64_t* off, int64_t* total) {
@@ -35,6 +36,9 @@ int layout(const gdn_layer_cfg_t* c, int64_t* off, int64_t* total) {
   sizes[GDN_WS_O_G] = 4;
   sizes[GDN_WS_QUANT] = (int64_t)gdn_quantize_workspace_size();
   sizes[GDN_WS_SCAN] = (int64_t)gdn_delta_rule_workspace_size(c->B, c->T, c->H, c->dk, c->dv);
+  sizes[GDN_WS_QKV_CONV] = c->conv ? M * NQKV * 2 : 0;
+  sizes[GDN_WS_G] = c->out_gate ? M * HV * 2 : 0;
+  sizes[GDN_WS_O_GATED] = c->out_gate ? M * HV * 2 : 0;
   int64_t pos = 0;
   for (int i = 0; i < GDN_WS_COUNT; ++i) {
     off[i] = pos;
@@ -77,6 +81,8 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
   if (!aligned(ws, 256)) return GDN_ERR_ALIGNMENT;
   if (!w->g_q || !w->g_k || !w->g_v || !w->g_a || !w->g_b || !w->g_out || !w->A_log || !w->dt_bias)
     return GDN_ERR_INVALID_ARG;
+  if ((cfg->conv && !w->conv_w) || (cfg->out_gate && (!w->g_g || !w->norm_w))) return GDN_ERR_INVALID_ARG;
+  if (cfg->conv && (NQKV % 8 != 0 || !aligned(w->conv_w, 16))) return GDN_ERR_UNSUPPORTED_SHAPE;
   if (M > 0) {
     if (!x || !y || !w->w_qkvab.codes || !w->w_qkvab.scales || !w->w_out.codes || !w->w_out.scales)
       return GDN_ERR_INVALID_ARG;
@@ -94,22 +100,38 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
   uint8_t* o_scales = base + off[GDN_WS_O_SCALES];
   float* o_g = reinterpret_cast<float*>(base + off[GDN_WS_O_G]);
   void* qws = base + off[GDN_WS_QUANT];
+  uint16_t* qkv_conv = reinterpret_cast<uint16_t*>(base + off[GDN_WS_QKV_CONV]);
+  uint16_t* g = reinterpret_cast<uint16_t*>(base + off[GDN_WS_G]);
+  uint16_t* o_gated = reinterpret_cast<uint16_t*>(base + off[GDN_WS_O_GATED]);
   const size_t qws_bytes = gdn_quantize_workspace_size();
   gdn_stream_t s = stream;
 
-  int st = gdn_quantize_nvfp4(x, GDN_DTYPE_BF16, M, D, D, GDN_QUANT_DYNAMIC, nullptr, x_codes, x_scales, GDN_SF_TILED, 0, x_g, qws,
-                              qws_bytes, s);
+  // x: its own amax (two passes), or the calibrated static scale (one pass)
+  int st = w->x_g_enc ? gdn_quantize_nvfp4(x, GDN_DTYPE_BF16, M, D, D, GDN_QUANT_GIVEN_SCALE, w->x_g_enc, x_codes,
+                                           x_scales, GDN_SF_TILED, 0, x_g, nullptr, 0, s)
+                      : gdn_quantize_nvfp4(x, GDN_DTYPE_BF16, M, D, D, GDN_QUANT_DYNAMIC, nullptr, x_codes, x_scales,
+                                           GDN_SF_TILED, 0, x_g, qws, qws_bytes, s);
   if (st) return st;
 
   gdn_nvfp4_t xa{x_codes, x_scales};
-  gdn_epilogue_segment_t seg[5] = {};
+  gdn_epilogue_segment_t seg[6] = {};
   seg[0] = {0, HK, GDN_EPI_STORE_BF16, w->g_q, qkv, NQKV, nullptr, nullptr};
   seg[1] = {HK, 2 * HK, GDN_EPI_STORE_BF16, w->g_k, qkv + HK, NQKV, nullptr, nullptr};
   seg[2] = {2 * HK, NQKV, GDN_EPI_STORE_BF16, w->g_v, qkv + 2 * HK, NQKV, nullptr, nullptr};
   seg[3] = {NQKV, NQKV + H, GDN_EPI_LOG_ALPHA, w->g_a, log_alpha, H, w->A_log, w->dt_bias};
   seg[4] = {NQKV + H, NQKV + 2 * H, GDN_EPI_BETA, w->g_b, beta, H, nullptr, nullptr};
-  st = gdn_gemm_nvfp4(&xa, x_g, &w->w_qkvab, M, NQKV + 2 * H, D, seg, 5, s);
+  if (cfg->out_gate) seg[5] = {NQKV + 2 * H, NQKV + 2 * H + HV, GDN_EPI_STORE_BF16, w->g_g, g, HV, nullptr, nullptr};
+  st = gdn_gemm_nvfp4(&xa, x_g, &w->w_qkvab, M, NQKV + 2 * H + (cfg->out_gate ? HV : 0), D, seg,
+                      cfg->out_gate ? 6 : 5, s);
   if (st) return st;
+
+  // the short convolution (+ SiLU) over the q | k | v channels, from zero history
+  const uint16_t* qkv_in = qkv;
+  if (cfg->conv) {
+    st = gdn_short_conv(qkv, cfg->B, cfg->T, NQKV, NQKV, w->conv_w, nullptr, qkv_conv, NQKV, nullptr, s);
+    if (st) return st;
+    qkv_in = qkv_conv;
+  }
 
   // Dynamic o scale: the scan records max |o| of the bf16 values it stores,
   // so o is quantized in one pass (given-amax mode) instead of amax pass +
@@ -119,14 +141,27 @@ int gdn_layer_fwd(const gdn_layer_weights_t* w, const gdn_layer_cfg_t* cfg, cons
   cudaError_t ce = cudaMemsetAsync(o_amax, 0, sizeof(unsigned), reinterpret_cast<cudaStream_t>(s));
   if (ce != cudaSuccess) return record_cuda_error(ce);
   OQuant oq{o_codes, o_scales, w->o_g_enc, o_g};
-  st = launch_delta_rule(qkv, qkv + HK, qkv + 2 * HK, NQKV, NQKV, NQKV, log_alpha, beta, S0, cfg->B, cfg->T, H, dk, dv,
-                         GDN_DR_L2NORM_QK, o, S_T, o_amax, reinterpret_cast<cudaStream_t>(s),
-                         w->o_g_enc ? &oq : nullptr);
+  const bool fuse_oq = w->o_g_enc && !cfg->out_gate;   // the scan quantizes o itself
+  st = launch_delta_rule(qkv_in, qkv_in + HK, qkv_in + 2 * HK, NQKV, NQKV, NQKV, log_alpha, beta, S0, cfg->B, cfg->T,
+                         H, dk, dv, GDN_DR_L2NORM_QK, o, S_T, cfg->out_gate ? nullptr : o_amax,
+                         reinterpret_cast<cudaStream_t>(s), fuse_oq ? &oq : nullptr, base + off[GDN_WS_SCAN],
+                         (size_t)gdn_delta_rule_workspace_size(cfg->B, cfg->T, H, dk, dv));
   if (st) return st;
 
-  if (!w->o_g_enc) {
-    st = gdn_quantize_nvfp4(o, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_GIVEN_AMAX, reinterpret_cast<const float*>(o_amax),
-                            o_codes, o_scales, GDN_SF_TILED, 0, o_g, nullptr, 0, s);
+  // the gated output norm; then o (or the gated o) is quantized for the
+  // output projection with its own amax or the static scale
+  const uint16_t* o_q = o;
+  if (cfg->out_gate) {
+    st = gdn_gated_rmsnorm(o, g, M, H, dv, w->norm_w, o_gated, reinterpret_cast<float*>(o_amax), s);
+    if (st) return st;
+    o_q = o_gated;
+  }
+  if (!fuse_oq) {
+    st = w->o_g_enc ? gdn_quantize_nvfp4(o_q, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_GIVEN_SCALE, w->o_g_enc, o_codes,
+                                         o_scales, GDN_SF_TILED, 0, o_g, nullptr, 0, s)
+                    : gdn_quantize_nvfp4(o_q, GDN_DTYPE_BF16, M, HV, HV, GDN_QUANT_GIVEN_AMAX,
+                                         reinterpret_cast<const float*>(o_amax), o_codes, o_scales, GDN_SF_TILED, 0,
+                                         o_g, nullptr, 0, s);
     if (st) return st;
   }
 

@@ -158,7 +158,36 @@ int launch_quantize_t(const E* x, int64_t rows, int64_t cols, int64_t ld, int mo
   return check_launch();
 }
 
+// *g_enc = 2688 / *amax (the per-tensor encode scale of a calibrated amax).
+__global__ void encode_scale_kernel(const float* __restrict__ amax, float* __restrict__ g_enc) {
+  *g_enc = encode_scale_from_amax(*amax);
+}
+
+template <typename In, typename E>
+int launch_amax_update_t(const E* x, int64_t rows, int64_t cols, int64_t ld, unsigned* amax_bits,
+                         cudaStream_t stream) {
+  if (rows == 0) return GDN_OK;
+  const int at = threads_for_row(cols / In::kPerVec);
+  dim3 grid;
+  grid_one_wave(amax_kernel<In, E>, rows, cols / In::kPerVec, at, grid);
+  amax_kernel<In, E><<<grid, at, 0, stream>>>(x, rows, cols / In::kPerVec, ld, amax_bits);
+  return check_launch();
+}
+
 }  // namespace
+
+int launch_amax_update(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, float* amax,
+                       cudaStream_t stream) {
+  unsigned* bits = reinterpret_cast<unsigned*>(amax);
+  if (x_dtype == GDN_DTYPE_F32)
+    return launch_amax_update_t<F32In>(static_cast<const float*>(x), rows, cols, ld, bits, stream);
+  return launch_amax_update_t<Bf16In>(static_cast<const uint16_t*>(x), rows, cols, ld, bits, stream);
+}
+
+int launch_encode_scale(const float* amax, float* g_enc, cudaStream_t stream) {
+  encode_scale_kernel<<<1, 1, 0, stream>>>(amax, g_enc);
+  return check_launch();
+}
 
 int launch_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, int mode,
                     const float* g_enc_in, uint8_t* codes, uint8_t* scales, int tiled, int64_t row_off, float* g_out,

@@ -27,12 +27,19 @@ Modules
   gates       decay gate log(alpha) and write strength beta
   delta_rule  sequential gated delta rule (the literal recurrence) and the
               chunked (UT / WY) form, both FP64
-  layer       the four steps composed into one layer forward
-  replay      clean vs NVFP4 trajectories of the recurrent state and the
-              decay of an impulse (the pages' robustness measurements)
+  layer       the four steps composed into one layer forward (optionally
+              with the short convolution and the gated output norm)
+  conv_norm   the short causal convolution + SiLU and the gated RMSNorm of
+              the Gated DeltaNet block (outside specification)
+  replay      clean vs NVFP4 trajectories of the recurrent state, the decay
+              of an impulse, gate-noise and gate-error-compression arms (the
+              pages' robustness measurements)
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
-against closed forms, brute force or independent library routines.  The
-values the replay harness reports are "parity unpinned": the pages' figures
-come from trained layers and real text; the harness itself is pinned.
+against closed forms, brute force, hand-worked examples or independent
+library routines; ``layer.layer_forward`` by a hand-worked two-token layer.
+Two things are "parity unpinned": the values the replay harness reports (the
+pages' figures come from trained layers and real text; the harness itself is
+pinned), and the composition of the layer's optional convolution and output
+gate (each step is pinned; their wiring has no hand-worked example).
 """

@@ -14,7 +14,12 @@ pinned (``tests/test_oracle_replay.py``) is the harness: zero error when
 nothing is quantized or no noise is added, the exact permutation invariance
 of the clean projections, an impulse on a write-free (beta = 0) trajectory
 decaying exactly as the product of the decays, and alpha noise on such a
-trajectory scaling each head's state by exactly prod (1 + sigma z).
+trajectory scaling each head's state by exactly prod (1 + sigma z) (by
+prod min(1 + sigma z, 1) when the perturbed decay is capped at 1 and every
+alpha is 1).  ``gate_error_compression`` (the page's account of how a
+projection error shrinks through the gates) is pinned by a single perturbed
+token whose gate errors are sigmoid(d) - 1/2 and the closed-form softplus
+difference.
 
 Readings where the pages are silent:
   * clean trajectory: FP64 projections of the bf16 activations with the FP32
@@ -139,9 +144,12 @@ def replay(d, seeds, checkpoints, t_imp, window, eps=0.01, quantize=True):
 
 def gate_noise_arm(scan_in, sigma, target, seeds, checkpoints, S0=None):
     """Multiplicative gate noise on a given trajectory: every alpha_t (target
-    "alpha") or beta_t ("beta") times (1 + sigma z), z ~ N(0, 1) per (token,
-    head), seeded.  Returns the relative state error against the noise-free
-    trajectory, [seeds, checkpoints]."""
+    "alpha" or "alpha_clamped") or beta_t ("beta") times (1 + sigma z),
+    z ~ N(0, 1) per (token, head), seeded.  "alpha" lets a perturbed decay
+    exceed 1 (the state then grows for that token); "alpha_clamped" caps it at
+    1, min(alpha_t (1 + sigma z), 1), so the noise can only make the state
+    forget faster or slower, never expand.  Returns the relative state error
+    against the noise-free trajectory, [seeds, checkpoints]."""
     q, k, v, la, be = scan_in
     S_ref = states_at(q, k, v, la, be, checkpoints, S0=S0)
     out = []
@@ -149,10 +157,31 @@ def gate_noise_arm(scan_in, sigma, target, seeds, checkpoints, S0=None):
         z = np.random.default_rng(s).standard_normal(la.shape)
         f = 1.0 + sigma * z
         assert np.all(f > 0), "noise too large for a multiplicative perturbation"
-        la_n, be_n = (la + np.log(f), be) if target == "alpha" else (la, be * f)
+        if target == "alpha":
+            la_n, be_n = la + np.log(f), be
+        elif target == "alpha_clamped":
+            la_n, be_n = np.minimum(la + np.log(f), 0.0), be
+        elif target == "beta":
+            la_n, be_n = la, be * f
+        else:
+            raise ValueError(f"unknown target {target!r}")
         S_n = states_at(q, k, v, la_n, be_n, checkpoints, S0=S0)
         out.append([rel_state_error(a, b) for a, b in zip(S_n, S_ref)])
     return np.asarray(out)
+
+
+def gate_error_compression(a_ref, b_ref, a_q, b_q, A_log, dt_bias):
+    """How an error on the gate projections shrinks through the gates
+    ("Anthology of the SOTA, theory-128", section "The account": the decay
+    and write gates pass the projection through softplus / exp and a sigmoid,
+    whose slopes are below 1 where the gates saturate).  Given reference and
+    perturbed projections a, b ([..., H]), returns the relative Frobenius
+    errors on a, on b, on 1 - alpha and on beta."""
+    la_r, be_r = gates(a_ref, b_ref, A_log, dt_bias)
+    la_q, be_q = gates(a_q, b_q, A_log, dt_bias)
+    oma_r, oma_q = -np.expm1(la_r), -np.expm1(la_q)       # 1 - alpha, without cancellation
+    return {"a": rel_state_error(a_q, a_ref), "b": rel_state_error(b_q, b_ref),
+            "one_minus_alpha": rel_state_error(oma_q, oma_r), "beta": rel_state_error(be_q, be_r)}
 
 
 def clean_scan_inputs(d):

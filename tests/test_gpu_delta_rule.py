@@ -142,3 +142,31 @@ def test_fp16_overflow_is_reported(mma_sync):
     o, S = _run(q, k, v, la, be, S0, mma_sync=mma_sync)
     o_ref, S_ref = delta_rule_chunked(q, k, v, la, be)
     assert rel_fro(o, o_ref) < TOL and rel_fro(S, S_ref) < TOL
+
+
+@pytest.mark.parametrize("T,H,o_fp32,s0", [(2000, 2, True, True), (4096, 4, False, False), (4100, 1, True, False)],
+                         ids=["ragged_s0", "bf16", "one_chain_ragged"])
+def test_segmented_scan_matches_oracle(T, H, o_fp32, s0):
+    """Few chains on long sequences: the library cuts each sequence into
+    segments (state transitions of the segments in parallel, their FP32
+    composition, then every segment from its entry state).  Same tolerance as
+    the unsegmented scan; the workspace query says the path is taken."""
+    assert _lib.lib().gdn_delta_rule_workspace_size(1, T, H, 128, 128) > 0
+    q, k, v, la, be, S0 = _case(1, T, H, 128, 128, 30 + T, with_s0=s0)
+    o, S = _run(q, k, v, la, be, S0, o_fp32=o_fp32)
+    o_ref, S_ref = delta_rule_chunked(q, k, v, la, be, S0=S0)
+    if not o_fp32:
+        from oracle.nvfp4 import round_bf16
+        o_ref = round_bf16(o_ref)
+    assert rel_fro(o, o_ref) < (TOL if o_fp32 else 3e-3)
+    assert rel_fro(S, S_ref) < TOL
+
+
+def test_segmented_scan_equals_unsegmented_within_tolerance():
+    """Without a workspace the same call runs every sequence in one piece."""
+    q, k, v, la, be, S0 = _case(1, 3000, 2, 128, 128, 77, with_s0=True)
+    args = (bf16_cuda(q), bf16_cuda(k), bf16_cuda(v), f32_cuda(la), f32_cuda(be))
+    o1, S1 = _lib.gdn_delta_rule_fwd(*args, S0=f32_cuda(S0), o_fp32=True)
+    o2, S2 = _lib.gdn_delta_rule_fwd(*args, S0=f32_cuda(S0), o_fp32=True, use_workspace=False)
+    _lib.stream_check()
+    assert rel_fro(to_np(o1), to_np(o2)) < TOL and rel_fro(to_np(S1), to_np(S2)) < TOL

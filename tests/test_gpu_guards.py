@@ -98,8 +98,9 @@ def test_gemm_stays_in_bounds_and_writes_everything(M, N, K, pitch):
 
 
 @pytest.mark.parametrize("B,T,H,d,mma_sync,o_fp32", [(2, 200, 2, 128, False, False), (1, 77, 3, 128, False, True),
-                                                    (2, 130, 2, 64, False, False), (1, 150, 2, 128, True, False)],
-                         ids=["tc_bf16", "tc_f32", "mma_sync_d64", "mma_sync_bf16"])
+                                                    (2, 130, 2, 64, False, False), (1, 150, 2, 128, True, False),
+                                                    (1, 2000, 2, 128, False, False)],
+                         ids=["tc_bf16", "tc_f32", "mma_sync_d64", "mma_sync_bf16", "tc_segmented"])
 def test_scan_stays_in_bounds_and_writes_everything(B, T, H, d, mma_sync, o_fp32):
     rng = np.random.default_rng(T)
     q = rng.standard_normal((B, T, H, d)).astype(np.float32)
@@ -155,7 +156,8 @@ def test_gates_stay_in_bounds_and_write_everything():
     assert _nan_free(la.t) and _nan_free(be.t)
 
 
-@pytest.mark.parametrize("dims", [(2, 200, 512, 4, 128, 128), (1, 96, 256, 2, 32, 32)], ids=["tc", "mma_sync"])
+@pytest.mark.parametrize("dims", [(2, 200, 512, 4, 128, 128), (1, 96, 256, 2, 32, 32), (1, 2048, 256, 2, 128, 128)],
+                         ids=["tc", "mma_sync", "tc_segmented"])
 def test_layer_stays_in_bounds_and_writes_everything(dims):
     """The layer's output, final state and workspace, each between canaries;
     y and S_T pre-filled with NaN."""

@@ -154,7 +154,8 @@ def test_layer_workload_sampled():
     (2, 200, 512, 4, 128, 128),    # tensor-core scan, 64-column d_v slices, ragged last chunk
     (2, 70, 512, 40, 128, 128),    # tensor-core scan, whole 128-column slices
     (1, 96, 256, 2, 32, 32),       # mma.sync scan: o quantized by a given-scale pass
-], ids=["tc_dvs64", "tc_dvs128", "mma_sync"])
+    (1, 2048, 256, 2, 128, 128),   # tensor-core scan in segments: o quantized in the last phase
+], ids=["tc_dvs64", "tc_dvs128", "mma_sync", "tc_segmented"])
 def test_layer_static_o_scale(dims):
     """A static encode scale for o (gdn_layer_weights_t.o_g_enc): the scan
     writes o's NVFP4 codes and scales itself.  Given the dynamic run's own

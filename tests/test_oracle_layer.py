@@ -97,3 +97,18 @@ def test_pin_catches_swapped_projections(golden_dir, swap):
     y, S_T, _ = layer_forward(x, Wq, A_log, dt_bias, H, DK, DV, S0=S0)
     assert _rel(y.reshape(T, D), g["y"]) > 0.05 or _rel(S_T.reshape(DK, DV), g["S_T"]) > 0.05
     assert _rel(y.reshape(T, D), g["y"]) > 1e-3
+
+
+def test_given_scales_equal_to_the_dynamic_ones_reproduce_the_example(golden_dir):
+    """Static activation scales: handing the layer the encode scales its two
+    activations would get dynamically (x: amax 1 -> 2688; o: amax 1.5 ->
+    1792) gives the same hand-worked result; another o scale changes y."""
+    g, s = _load(golden_dir)
+    x, W, A_log, dt_bias, S0 = _inputs(g, s)
+    Wq = quantize_weights(W)
+    y, S_T, inter = layer_forward(x, Wq, A_log, dt_bias, H, DK, DV, S0=S0, x_g_enc=np.float32(2688.0),
+                                  o_g_enc=np.float32(1792.0))
+    np.testing.assert_array_equal(y.reshape(T, D), g["y"])
+    assert inter["oq"]["g_enc"] == np.float32(1792.0) and inter["xq"]["g_enc"] == np.float32(2688.0)
+    y2, _, _ = layer_forward(x, Wq, A_log, dt_bias, H, DK, DV, S0=S0, o_g_enc=np.float32(1792.0 * 3.3))
+    assert _rel(y2.reshape(T, D), g["y"]) > 1e-3
