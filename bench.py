@@ -173,9 +173,11 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    W = WORKLOAD
+    W = dict(WORKLOAD, B=args.layer_B, T=args.layer_T)
     B, T, D, H, dk, dv = W["B"], W["T"], W["d_model"], W["H"], W["dk"], W["dv"]
     M, HK, HV = B * T, H * dk, H * dv
+    workload_name = (WORKLOAD_NAME if (B, T) == (WORKLOAD["B"], WORKLOAD["T"]) else
+                     f"gdn_w4a4_layer_prefill B={B} T={T} d_model={D} H={H} dk=dv={dk} (reduced: a profiling case)")
     d = inputs.layer_inputs(B, T, D, H, dk, dv, seed=replica_seed(rank))
     stream = torch.cuda.current_stream()
     lw = _lib.QuantizedLayerWeights(d["W"], d["A_log"], d["dt_bias"], H, dk, dv, device=dev)
@@ -401,7 +403,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3, fp32 acc); scan fp16 mma, fp32 state",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAME, **W, "tokens_per_step_per_gpu": M,
+        "config": {"workload": workload_name, **W, "tokens_per_step_per_gpu": M,
                    "l2": "inputs exceed L2 (x 335 MB, q/k/v 805 MB per step); no flush",
                    "parallelism": f"replicas x{world} (independent batches per GPU)"},
         "e2e": {"value": round(tokens_per_step / (e2e_ms / 1e3), 1), "unit": UNIT,
@@ -741,6 +743,10 @@ def main():
                     help="tokens of the oracle sample (CPU baseline and --impl reference)")
     ap.add_argument("--only", choices=["gemm", "scan"], default=None,
                     help="time only the standalone GEMM or scan workload (profiling target)")
+    ap.add_argument("--layer-B", type=int, default=WORKLOAD["B"],
+                    help="sequences of the layer workload (a smaller value gives a profiling case)")
+    ap.add_argument("--layer-T", type=int, default=WORKLOAD["T"],
+                    help="tokens per sequence of the layer workload (a smaller value gives a profiling case)")
     ap.add_argument("--replay", action="store_true",
                     help="run the replay workload (state error of NVFP4 trajectories, impulse, gate errors)")
     args = ap.parse_args()
