@@ -335,7 +335,8 @@ int gdn_delta_rule_step(const void* q, const void* k, const void* v,
  * gdn_gated_rmsnorm: per (token m, head h) row of dv values of o and g
  *   (bf16 [M, H*dv], row m*H + h at (m*H + h)*dv):
  *     y = o / sqrt(mean(o^2) + 1e-6) * gamma * SiLU(g)          (bf16 out)
- *   gamma FP32 [dv]; dv in {32, 64, 128}.  When amax is non-NULL, max |y|
+ *   o, g, y 16-byte aligned; gamma FP32 [dv]; dv in {32, 64, 128}.  When
+ *   amax is non-NULL, max |y|
  *   (of the stored bf16 values) is folded into *amax (>= 0 on entry), for a
  *   given-amax quantization of y.
  * ------------------------------------------------------------------------ */

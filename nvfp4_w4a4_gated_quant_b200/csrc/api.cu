@@ -236,7 +236,7 @@ int gdn_gated_rmsnorm(const void* o, const void* g, int64_t M, int H, int dv, co
   if (M < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
   if (dv != 32 && dv != 64 && dv != 128) return GDN_ERR_UNSUPPORTED_SHAPE;
   if (M > 0 && (!o || !g || !gamma || !y)) return GDN_ERR_INVALID_ARG;
-  if ((o && !aligned(o, 2)) || (g && !aligned(g, 2)) || (y && !aligned(y, 2)) || (amax && !aligned(amax, 4)))
+  if ((o && !aligned(o, 16)) || (g && !aligned(g, 16)) || (y && !aligned(y, 16)) || (amax && !aligned(amax, 4)))
     return GDN_ERR_ALIGNMENT;
   return launch_gated_rmsnorm(static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(g), M, H, dv, gamma,
                               static_cast<uint16_t*>(y), amax, as_stream(stream));
