@@ -401,7 +401,10 @@ __device__ __forceinline__ void pipe_load_v(uint32_t sb, uint64_t* bar, const Ma
 }
 
 // In place: the bf16 rows r0 .. r0+63 of [K; Q] -> L2-normalised FP16
-// (256 threads, four per row, 32 columns each).
+// (256 threads, four per row, 32 columns each).  Thread pq of a row takes the
+// 16-byte chunks pq and pq + 4 of both 64-column atoms, in an order that puts
+// the eight threads of two adjacent rows on eight distinct swizzled bank
+// groups (the plain column order hit every bank group twice).
 template <int DVS>
 __device__ __forceinline__ void pipe_normalize(uint32_t t3, int r0, int tid, int l2norm, float& hmax) {
   using M = PMap<DVS>;
@@ -411,8 +414,8 @@ __device__ __forceinline__ void pipe_normalize(uint32_t t3, int r0, int tid, int
   uint32_t off[QC / 8];
 #pragma unroll
   for (int i = 0; i < QC / 8; ++i) {
-    const int col = pq * QC + 8 * i;
-    off[i] = t3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(r0 + pr, col & 63);
+    const int L = pq + 4 * ((i & 1) ^ (pr & 1));   // eight distinct bank groups per two rows
+    off[i] = t3 + (uint32_t)(i >> 1) * M::T3_ATOM + swz(r0 + pr, 8 * L);
     unpack_bf16x8(ld_s128(off[i]), &v[8 * i]);
   }
   float s0 = 0.f, s1 = 0.f;
@@ -724,12 +727,14 @@ __global__ void __launch_bounds__(NTP, 1)
       } else {
         // ---- beside the inverse: Q' = diag(e^{G_t}) Q in place (warps 4-7;
         // MMA-a has finished reading Q)
+        // (the two threads of a row walk their atoms half a row apart, so
+        // four rows' eight chunks fall on distinct bank groups)
         const int j = tid - 128;
         const int row = j >> 1, c0 = (j & 1) * 64;
         const float e = eg[row];
 #pragma unroll
         for (int cc = 0; cc < 64; cc += 8) {
-          const int col = c0 + cc;
+          const int col = c0 + ((cc + 32 * (j & 1)) & 63);
           scale_chunk_h(t3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(64 + row, col & 63), e);
         }
       }
@@ -870,10 +875,11 @@ __global__ void __launch_bounds__(NTP, 1)
       // c+2's k and q as soon as MMA-1 completes
       {
         const float* dkf = fb + Fac::DKF;
-        const int row = gt >> 1, half = gt & 1;
+        const int row = gt >> 1, half = gt & 1;     // halves half a row apart: distinct bank groups
         const float e = dkf[row];
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 8) {
+        for (int c8 = 0; c8 < 64; c8 += 8) {
+          const int cc = (c8 + 32 * half) & 63;
           float f[8];
           unpack_h8(ld_s128(t3 + (uint32_t)half * M::T3_ATOM + swz(row, cc)), f);
 #pragma unroll
