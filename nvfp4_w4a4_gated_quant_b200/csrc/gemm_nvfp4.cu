@@ -301,7 +301,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   SegSmem* segs = reinterpret_cast<SegSmem*>(staging + STAGING_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(segs + GDN_MAX_SEGMENTS);
   uint64_t* empty = full + STAGES;
-  uint64_t* pfull = empty + STAGES;        // [STAGES] pair, CTA 0: the peer's half of a stage has landed
+  uint64_t* pfull = empty + STAGES;        // [STAGES] pair, CTA 0: stage s of both CTAs is ready (see below)
   uint64_t* sf_land = pfull + STAGES;      // [STAGES] a stage's scale copies have landed
   uint64_t* sf_full = sf_land + STAGES;    // [SF_NBUF] a TMEM scale buffer is filled
   uint64_t* sf_free = sf_full + SF_NBUF;   // [SF_NBUF] the MMAs that read a buffer are done
@@ -321,7 +321,11 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&pfull[s], 1);
+      // a pair's MMA warp waits on one barrier per k-block (each check costs
+      // the issuing warp ~150 cycles): CTA 0's own operand tiles complete on
+      // it (its producer's arrive.expect_tx), plus the peer's relay and the
+      // eight scale loaders of both CTAs
+      mbar_init(&pfull[s], 10);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_land[s], 1);
     }
@@ -381,6 +385,9 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     // ------------------------------------------------------- producer
     // The whole warp runs this loop; one elected lane issues each copy.
     uint32_t it = 0;   // k-blocks issued
+    // the barrier the operand tiles complete on: CTA 0 of a pair counts them
+    // into the MMA warp's one barrier
+    uint64_t* opbar = PAIR && rank == 0 ? pfull : full;
     bool ok = true;
     for (int tile = cid; ok && tile < p.num_tiles; tile += ncl) {
       const int mb = tile / p.num_n, nb = tile % p.num_n;
@@ -397,9 +404,9 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         const uint32_t round = it / STAGES;
         if (!wait_or_abort(&empty[s], (round & 1) ^ 1, p.status, abort_flag)) { ok = false; break; }
         const int nks = min(BK / KSTEP, ksteps_total - kb * (BK / KSTEP));
-        mbar_arrive_expect_tx_warp(&full[s], (a_live ? A_BYTES : 0) + (b_live ? S::B_CTA_BYTES : 0));
-        if (a_live) tma_load_2d_warp(sA + s * A_BYTES, &tmap_a, &full[s], kb * (BK / 2), a_row);
-        if (b_live) tma_load_2d_warp(sB + s * S::B_CTA_BYTES, &tmap_b, &full[s], kb * (BK / 2), b_row);
+        mbar_arrive_expect_tx_warp(&opbar[s], (a_live ? A_BYTES : 0) + (b_live ? S::B_CTA_BYTES : 0));
+        if (a_live) tma_load_2d_warp(sA + s * A_BYTES, &tmap_a, &opbar[s], kb * (BK / 2), a_row);
+        if (b_live) tma_load_2d_warp(sB + s * S::B_CTA_BYTES, &tmap_b, &opbar[s], kb * (BK / 2), b_row);
         // the stage's scales after its operand tiles (248 -> 246 us)
         mbar_arrive_expect_tx_warp(&sf_land[s], (uint32_t)nks * 512u * ((a_live ? 1u : 0u) + (uint32_t)nh));
         if (a_live)
@@ -415,7 +422,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
     // (it - 1 - s) / STAGES).
     for (uint32_t s = 0; s < (uint32_t)STAGES && s < it; ++s) {
       const uint32_t last_round = (it - 1 - s) / STAGES;
-      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&full[s], last_round & 1); ++i) __nanosleep(32);
+      for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&opbar[s], last_round & 1); ++i) __nanosleep(32);
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(&sf_land[s], last_round & 1); ++i) __nanosleep(32);
     }
     __syncwarp();
@@ -470,7 +477,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
         __syncwarp();
         if (lane == 0) {
           if (PAIR)
-            mbar_arrive_cluster(cluster_addr(&sf_full[buf], 0));
+            mbar_arrive_cluster(cluster_addr(&pfull[buf], 0));   // buf == stage in a pair
           else
             mbar_arrive(&sf_full[buf]);
         }
@@ -503,9 +510,9 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t buf = it % NBUF;
-        if (!wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag) ||
-            (PAIR && !wait_or_abort(&pfull[s], (it / STAGES) & 1, p.status, abort_flag)) ||
-            !wait_or_abort(&sf_full[buf], (it / NBUF) & 1, p.status, abort_flag)) {
+        if (PAIR ? !wait_or_abort(&pfull[s], (it / STAGES) & 1, p.status, abort_flag)
+                 : (!wait_or_abort(&full[s], (it / STAGES) & 1, p.status, abort_flag) ||
+                    !wait_or_abort(&sf_full[buf], (it / NBUF) & 1, p.status, abort_flag))) {
           ok = false;
           break;
         }
