@@ -10,7 +10,8 @@
 //   out    = o / sqrt(mean_dv(o^2) + 1e-6) * gamma * SiLU(g)   per (token, head)
 // Both are HBM-bound elementwise passes: FP32 arithmetic on bf16 storage,
 // 8- and 16-byte vectors with several rows in flight per thread, one thread
-// per four channels (convolution) or DV/8 lanes per (token, head) row (norm).  SiLU(u) = u sigmoid(u) with
+// per four channels (convolution) or DV/8 lanes per (token, head) row
+// (norm).  SiLU(u) = u sigmoid(u) with
 // sigmoid(u) = 1/2 + tanh(u/2)/2 on the SFU's tanh.approx (relative error
 // ~2^-11, below the bf16 rounding of the stored result), so the passes stay
 // memory-bound.
@@ -25,7 +26,7 @@ namespace {
 constexpr int CW = 4;          // kernel width
 constexpr int CONV_TOK = 64;   // tokens one thread walks
 constexpr int CONV_THREADS = 256;
-constexpr int CONV_NR = 8;     // input rows in flight per thread
+constexpr int CONV_NR = 4;     // input rows per group; two groups in flight
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -59,7 +60,7 @@ __device__ __forceinline__ uint2 pack4(const float* f) {
 
 // grid (channel quads / CONV_THREADS, token blocks, batch): a thread keeps
 // the three previous inputs of its four channels in registers while it walks
-// CONV_TOK tokens, reading each input row once with CONV_NR rows in flight.
+// CONV_TOK tokens, reading each input row once, in groups of CONV_NR rows.
 __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t C,
                                                                   int64_t ld_x, const float* __restrict__ w,
                                                                   const uint16_t* __restrict__ state_in,
@@ -106,13 +107,27 @@ __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const uint16_t
     }
     *reinterpret_cast<uint2*>(y + (b * T + t) * ld_y + c0) = pack4(out);
   };
+  // groups of CONV_NR rows: the next group's loads are issued before this
+  // group's arithmetic and stores
   int64_t t = t_begin;
+  uint2 cur[CONV_NR], nxt[CONV_NR];
+  if (t + CONV_NR <= t_end) {
+#pragma unroll
+    for (int u = 0; u < CONV_NR; ++u) cur[u] = *reinterpret_cast<const uint2*>(x + (b * T + t + u) * ld_x + c0);
+  }
   for (; t + CONV_NR <= t_end; t += CONV_NR) {
-    uint2 raw[CONV_NR];
+    const bool more = t + 2 * CONV_NR <= t_end;
+    if (more) {
 #pragma unroll
-    for (int u = 0; u < CONV_NR; ++u) raw[u] = *reinterpret_cast<const uint2*>(x + (b * T + t + u) * ld_x + c0);
+      for (int u = 0; u < CONV_NR; ++u)
+        nxt[u] = *reinterpret_cast<const uint2*>(x + (b * T + t + CONV_NR + u) * ld_x + c0);
+    }
 #pragma unroll
-    for (int u = 0; u < CONV_NR; ++u) step(raw[u], t + u);
+    for (int u = 0; u < CONV_NR; ++u) step(cur[u], t + u);
+    if (more) {
+#pragma unroll
+      for (int u = 0; u < CONV_NR; ++u) cur[u] = nxt[u];
+    }
   }
   for (; t < t_end; ++t) step(*reinterpret_cast<const uint2*>(x + (b * T + t) * ld_x + c0), t);
   // the last three inputs (carried state included) for the next call
