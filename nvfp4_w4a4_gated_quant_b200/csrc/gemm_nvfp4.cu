@@ -555,7 +555,7 @@ gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_const
       for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(mma_done, 0); ++i) __nanosleep(32);
     }
     __syncwarp();
-  } else if (warp >= EPI_WARP0) {
+  } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + NUM_EPI_WARPS) {
     // --------------------------------------------------------- epilogue
     const int ew = warp - EPI_WARP0;
     const int quad = warp & 3;            // TMEM lanes quad*32 .. quad*32+31
