@@ -637,9 +637,12 @@ __global__ void __launch_bounds__(NTP, 1)
       if (warp < 4) {
         // ---- X = (I + L)^{-1} and Xw = X diag(beta_s e^{G_{s-1}}) (warps 0-3)
         const float* d1 = fb + Fac::D1;
-        if (lane < 16) {
+        {
+          // every lane solves column j = lane % 16 (the two half-warps the
+          // same column): lanes 0-15 store X, lanes 16-31 store Xw
           const int base = 16 * warp;
-          const int j = lane;
+          const int j = lane & 15;
+          const bool wside = lane >= 16;
           const float4* lb4 = reinterpret_cast<const float4*>(smem + M::LD32 + warp * 1024);
           float acc[16];
 #pragma unroll
@@ -660,18 +663,16 @@ __global__ void __launch_bounds__(NTP, 1)
             }
             acc[t] = (t < j) ? 0.0f : (p0 + p1) + (p2 + p3);
           }
-          const float dj = d1[base + j];
-          __syncwarp(0x0000ffffu);
+          const float dj = wside ? d1[base + j] : 1.0f;
+          const uint32_t dst = wside ? Xwb : Xb;
+          __syncwarp();
           float am = 0.0f;
 #pragma unroll
           for (int t = 0; t < 16; ++t) {
-            const float xw = acc[t] * dj;
-            am = fmaxf(am, fmaxf(fabsf(acc[t]), fabsf(xw)));
-            const __half hx = __float2half_rn(acc[t]);
-            const __half hw = __float2half_rn(xw);
-            asm volatile("st.shared.b16 [%0], %1;" ::"r"(Xb + swz(base + t, base + j)), "h"(__half_as_ushort(hx))
-                         : "memory");
-            asm volatile("st.shared.b16 [%0], %1;" ::"r"(Xwb + swz(base + t, base + j)), "h"(__half_as_ushort(hw))
+            const float x = acc[t] * dj;
+            am = fmaxf(am, fabsf(x));
+            const __half hx = __float2half_rn(x);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(dst + swz(base + t, base + j)), "h"(__half_as_ushort(hx))
                          : "memory");
           }
           hmax = fmaxf(hmax, am);
