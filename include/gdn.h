@@ -266,7 +266,16 @@ int gdn_gates(const float* a, const float* b, int64_t M, int H,
  * tensor cores (tcgen05.mma, state kept in TMEM); other shapes, or the flag
  * GDN_DR_MMA_SYNC, run the warp-level mma.sync kernel.  Both compute the same
  * chunk form; they differ in FP32 summation order only.
- * ws     gdn_delta_rule_workspace_size(...) bytes (may be 0 / NULL).
+ * ws     gdn_delta_rule_workspace_size(...) bytes (may be 0 / NULL), 256-byte
+ *        aligned, owned by the caller, not read after the call's kernels
+ *        end.  The tensor-core path uses it when it cuts long sequences on
+ *        few chains into segments (the size is 0 otherwise): (1) the segment
+ *        states, then (2) 16 KB per chunk of 64 tokens per (batch, head): the
+ *        inverse (I + L)^{-1} of every chunk and its beta-weighted copy,
+ *        computed once by a wide pass ahead of both passes over the
+ *        segments.  With fewer bytes than (1) + (2) both passes invert each
+ *        chunk themselves (the same bits), with fewer than (1) every sequence
+ *        runs in one piece.  Unused by the mma.sync kernel.
  * flags  GDN_DR_L2NORM_QK | GDN_DR_O_FP32 | GDN_DR_MMA_SYNC; any other bit
  *        (GDN_DR_DECAYED_READ included: the chunked form implements the
  *        literal read) is GDN_ERR_INVALID_ARG.

@@ -41,6 +41,7 @@ namespace {
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kImgBytes = 128 * 128;   // one chunk's [Xw; X]: 128 rows of 64 FP16
 
 // Per-token factors of one chunk (float offsets into a factor block): G_t and
 // G_{t-1} times log2(e), beta_t, beta_t e^{G_{t-1}}, e^{G_t}, e^{G_C - G_t}, and
@@ -97,6 +98,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Untiled bulk copy global -> shared (16-byte aligned, size % 16 == 0),
+// completing on the mbarrier at shared address bar.
+__device__ __forceinline__ void bulk_load_s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int32_t c0, int32_t c1,
                                             int32_t c2) {
   asm volatile(
@@ -195,6 +203,11 @@ struct Args {
   float* S_T;
   unsigned* o_amax;
   int* status;
+  // [Xw; X] images of every chunk, precomputed by chunk_inverse_kernel
+  // (kernels instantiated with XPRE), indexed ((b * nch_T + chunk) * H + h);
+  // nch_T = chunks per sequence
+  const uint8_t* xinv;
+  int64_t nch_T;
   // fused NVFP4 quantization of the bf16 o (codes == nullptr: off)
   uint8_t* oq_codes;
   uint8_t* oq_scales;
@@ -372,9 +385,10 @@ __device__ __forceinline__ void scale_chunk_h(uint32_t addr, float e) {
   st_chunk_h(addr, f);
 }
 
-// The q and k rows of chunk t0 into stage s, and (separately) its v rows;
-// rows past the end of the sequence arrive as zeros.  One thread each; the
-// stage's load barrier completes once both halves have landed.
+// The q and k rows of chunk t0 into stage s, and (separately) its v rows
+// (with XPRE also the chunk's precomputed [Xw; X]); rows past the end of the
+// sequence arrive as zeros.  One thread each; the stage's load barrier
+// completes once both halves have landed.
 template <int DVS>
 __device__ __forceinline__ void pipe_load_kq(uint32_t sb, uint64_t* bar, const Maps& m, int b, int h, int64_t t0,
                                              int s) {
@@ -388,26 +402,30 @@ __device__ __forceinline__ void pipe_load_kq(uint32_t sb, uint64_t* bar, const M
     tma_load_3d(t3 + at * M::T3_ATOM + 64 * 128, &m.q, bar_s, h * DK + 64 * at, (int32_t)t0, b);
   }
 }
-template <int DVS>
+template <int DVS, bool XPRE>
 __device__ __forceinline__ void pipe_load_v(uint32_t sb, uint64_t* bar, const Maps& m, const Args& a, int b, int h,
                                             int dv_off, int64_t t0, int s) {
   using M = PMap<DVS>;
-  mbar_arrive_expect_tx(bar, M::LD_V);
+  mbar_arrive_expect_tx(bar, M::LD_V + (XPRE ? kImgBytes : 0u));
   const uint32_t bar_s = smem_u32(bar);
   const uint32_t vb = sb + M::vb(s);
 #pragma unroll
   for (int at = 0; at < DVS / 64; ++at)
     tma_load_3d(vb + at * 8192, &m.v, bar_s, h * a.dv + dv_off + 64 * at, (int32_t)t0, b);
+  // the chunk's precomputed [Xw; X] into rows 64..191 of [A; Xw; X]
+  if (XPRE)
+    bulk_load_s(sb + M::pt(s) + 64 * 128, a.xinv + (((int64_t)b * a.nch_T + t0 / C) * a.H + h) * kImgBytes,
+                kImgBytes, bar_s);
 }
 
-// In place: the bf16 rows r0 .. r0+63 of [K; Q] -> L2-normalised FP16
-// (256 threads, four per row, 32 columns each).  Thread pq of a row takes the
+// In place: the bf16 rows r0 .. r0+nthreads/4-1 of a tile of 64-column atoms
+// ATOM bytes apart -> L2-normalised FP16 (four threads per row, 32 columns
+// each).  Thread pq of a row takes the
 // 16-byte chunks pq and pq + 4 of both 64-column atoms, in an order that puts
 // the eight threads of two adjacent rows on eight distinct swizzled bank
 // groups (the plain column order hit every bank group twice).
-template <int DVS>
-__device__ __forceinline__ void pipe_normalize(uint32_t t3, int r0, int tid, int l2norm, float& hmax) {
-  using M = PMap<DVS>;
+template <uint32_t ATOM>
+__device__ __forceinline__ void normalize_rows(uint32_t t3, int r0, int tid, int l2norm, float& hmax) {
   constexpr int QC = DK / 4;
   const int pr = tid >> 2, pq = tid & 3;
   float v[QC];
@@ -415,7 +433,7 @@ __device__ __forceinline__ void pipe_normalize(uint32_t t3, int r0, int tid, int
 #pragma unroll
   for (int i = 0; i < QC / 8; ++i) {
     const int L = pq + 4 * ((i & 1) ^ (pr & 1));   // eight distinct bank groups per two rows
-    off[i] = t3 + (uint32_t)(i >> 1) * M::T3_ATOM + swz(r0 + pr, 8 * L);
+    off[i] = t3 + (uint32_t)(i >> 1) * ATOM + swz(r0 + pr, 8 * L);
     unpack_bf16x8(ld_s128(off[i]), &v[8 * i]);
   }
   float s0 = 0.f, s1 = 0.f;
@@ -434,7 +452,146 @@ __device__ __forceinline__ void pipe_normalize(uint32_t t3, int r0, int tid, int
   for (int i = 0; i < QC / 8; ++i) st_chunk_hc(off[i], &v[8 * i], hmax);
 }
 
-template <int DVS, bool O_F32>
+// One row t of L (quarters 0 and 1 of the K K^T accumulator: rows t < 64),
+// columns s0 = 32 colhalf .. s0 + 31 in r:
+//   L_ts = beta_t e^{G_{t-1} - G_s} k_t.k_s  (s < t),  0 otherwise,
+// stored as FP16 in X's place (the inverse overwrites it), the row's chunks of
+// Xw zeroed (the inverse writes only Xw's lower blocks, and the rows may hold
+// other data), and the row's piece of its diagonal 16 x 16 block kept in FP32
+// at ld32 (4 blocks of 16 x 16).
+__device__ __forceinline__ void build_l_row(const uint32_t (&r)[32], int t, int colhalf, uint32_t Xb, uint32_t Xwb,
+                                            uint32_t ld32, const float* be, const float* g2m1, const float* g2,
+                                            float& hmax) {
+  const int s0 = colhalf * 32;
+  const float bt = be[t], gm = g2m1[t];
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int s2 = s0 + i;
+    v[i] = (s2 < t) ? bt * ex2(fminf(gm - g2[s2], 0.0f)) * __uint_as_float(r[i]) : 0.0f;
+  }
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    st_chunk_hc(Xb + swz(t, s0 + 8 * cc), &v[8 * cc], hmax);
+    st_s128(Xwb + swz(t, s0 + 8 * cc), 0u, 0u, 0u, 0u);
+  }
+  const int blk = t >> 4;
+  if ((blk >> 1) == colhalf) {
+    // the diagonal block's 16 columns are the first or second half of these 32
+    const uint32_t dst = ld32 + (uint32_t)(blk * 256 + (t & 15) * 16) * 4;
+    if (blk & 1) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        st_s128(dst + cc * 16, __float_as_uint(v[16 + 4 * cc]), __float_as_uint(v[17 + 4 * cc]),
+                __float_as_uint(v[18 + 4 * cc]), __float_as_uint(v[19 + 4 * cc]));
+    } else {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        st_s128(dst + cc * 16, __float_as_uint(v[4 * cc]), __float_as_uint(v[1 + 4 * cc]),
+                __float_as_uint(v[2 + 4 * cc]), __float_as_uint(v[3 + 4 * cc]));
+    }
+  }
+}
+
+// X = (I + L)^{-1} and Xw = X diag(d1) (d1_s = beta_s e^{G_{s-1}}), both
+// FP16 in 128-byte-swizzled 64 x 64 tiles, from L in X's place and its FP32
+// diagonal blocks at ld32.  Four warps (warp = 0..3, 128 threads meeting at
+// named barrier bar_id): the diagonal 16 x 16 blocks by substitution in FP32,
+// then the off-diagonal blocks level by level on mma.sync,
+//   X_ij = -X_ii sum_{i > k >= j} L_ik X_kj.
+__device__ __forceinline__ void chunk_inverse(const float4* ld32, uint32_t Xb, uint32_t Xwb, const float* d1,
+                                              int warp, int lane, float& hmax, int bar_id) {
+  {
+    // every lane solves column j = lane % 16 (the two half-warps the
+    // same column): lanes 0-15 store X, lanes 16-31 store Xw
+    const int base = 16 * warp;
+    const int j = lane & 15;
+    const bool wside = lane >= 16;
+    const float4* lb4 = ld32 + warp * 64;
+    float acc[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float l[16];
+#pragma unroll
+      for (int cc = 0; cc < (t + 3) / 4; ++cc) {
+        const float4 v4 = lb4[t * 4 + cc];
+        l[4 * cc] = v4.x; l[4 * cc + 1] = v4.y; l[4 * cc + 2] = v4.z; l[4 * cc + 3] = v4.w;
+      }
+      float p0 = (t == j) ? 1.0f : 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
+#pragma unroll
+      for (int s2 = 0; s2 < t; ++s2) {
+        if ((s2 & 3) == 0) p0 = fmaf(-l[s2], acc[s2], p0);
+        if ((s2 & 3) == 1) p1 = fmaf(-l[s2], acc[s2], p1);
+        if ((s2 & 3) == 2) p2 = fmaf(-l[s2], acc[s2], p2);
+        if ((s2 & 3) == 3) p3 = fmaf(-l[s2], acc[s2], p3);
+      }
+      acc[t] = (t < j) ? 0.0f : (p0 + p1) + (p2 + p3);
+    }
+    const float dj = wside ? d1[base + j] : 1.0f;
+    const uint32_t dst = wside ? Xwb : Xb;
+    __syncwarp();
+    float am = 0.0f;
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const float x = acc[t] * dj;
+      am = fmaxf(am, fabsf(x));
+      const __half hx = __float2half_rn(x);
+      asm volatile("st.shared.b16 [%0], %1;" ::"r"(dst + swz(base + t, base + j)), "h"(__half_as_ushort(hx))
+                   : "memory");
+    }
+    hmax = fmaxf(hmax, am);
+  }
+  named_bar(bar_id, 128);
+  uint32_t Pk[3][4];
+  const int g = lane >> 2, c4 = lane & 3;
+  {
+    uint32_t af[4];
+    frag_a(af, Xb, 16 * warp, 16 * warp, lane);
+#pragma unroll
+    for (int dd = 1; dd <= 3; ++dd) {
+      if (dd <= warp) {
+        float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t bf[4];
+        frag_b_kn(bf, Xb, 16 * warp, 16 * (warp - dd), lane);   // still L_ik
+        mma16816(p0, af, bf[0], bf[1]);
+        mma16816(p1, af, bf[2], bf[3]);
+        c_to_a(Pk[dd - 1], p0, p1);
+      }
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int d = 1; d < 4; ++d) {
+    if (warp >= d) {
+      const int i = warp, jb = warp - d;
+      float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int dd = 1; dd <= 3; ++dd) {
+        if (dd <= d) {
+          uint32_t bf[4];
+          frag_b_kn(bf, Xb, 16 * (i - dd), 16 * jb, lane);
+          mma16816(z0, Pk[dd - 1], bf[0], bf[1]);
+          mma16816(z1, Pk[dd - 1], bf[2], bf[3]);
+        }
+      }
+      const int r0 = 16 * i + g, cc = 16 * jb + 2 * c4;
+      const float da = d1[cc], db = d1[cc + 1], dc = d1[cc + 8], dd2 = d1[cc + 9];
+      hmax = fmaxf(hmax, fmaxf(fmaxf(fmaxf(fabsf(z0[0]), fabsf(z0[1])), fmaxf(fabsf(z0[2]), fabsf(z0[3]))),
+                               fmaxf(fmaxf(fabsf(z1[0]), fabsf(z1[1])), fmaxf(fabsf(z1[2]), fabsf(z1[3])))));
+      st_s32(Xb + swz(r0, cc), pack_h2(-z0[0], -z0[1]));
+      st_s32(Xb + swz(r0 + 8, cc), pack_h2(-z0[2], -z0[3]));
+      st_s32(Xb + swz(r0, cc + 8), pack_h2(-z1[0], -z1[1]));
+      st_s32(Xb + swz(r0 + 8, cc + 8), pack_h2(-z1[2], -z1[3]));
+      st_s32(Xwb + swz(r0, cc), pack_h2(-z0[0] * da, -z0[1] * db));
+      st_s32(Xwb + swz(r0 + 8, cc), pack_h2(-z0[2] * da, -z0[3] * db));
+      st_s32(Xwb + swz(r0, cc + 8), pack_h2(-z1[0] * dc, -z1[1] * dd2));
+      st_s32(Xwb + swz(r0 + 8, cc + 8), pack_h2(-z1[2] * dc, -z1[3] * dd2));
+    }
+    named_bar(bar_id, 128);
+  }
+}
+
+template <int DVS, bool O_F32, bool XPRE>
 __global__ void __launch_bounds__(NTP, 1)
     delta_rule_pipe_kernel(const __grid_constant__ Args a, const __grid_constant__ Maps maps) {
   using M = PMap<DVS>;
@@ -515,12 +672,12 @@ __global__ void __launch_bounds__(NTP, 1)
   if (tid == LD_ISSUER) {
     if (nchunks > 0) {
       pipe_load_kq<DVS>(sb, &bar_ld[0], maps, b, h, seg0, 0);
-      pipe_load_v<DVS>(sb, &bar_ld[0], maps, a, b, h, dv_off, seg0, 0);
+      pipe_load_v<DVS, XPRE>(sb, &bar_ld[0], maps, a, b, h, dv_off, seg0, 0);
       kq0 = v0 = 1;
     }
     if (nchunks > 1) {
       pipe_load_kq<DVS>(sb, &bar_ld[1], maps, b, h, seg0 + C, 1);
-      pipe_load_v<DVS>(sb, &bar_ld[1], maps, a, b, h, dv_off, seg0 + C, 1);
+      pipe_load_v<DVS, XPRE>(sb, &bar_ld[1], maps, a, b, h, dv_off, seg0 + C, 1);
       kq1 = v1 = 1;
     }
   }
@@ -552,8 +709,8 @@ __global__ void __launch_bounds__(NTP, 1)
       }
       if (!grp_wait(&bar_ld[s], ph, abort_flag, a.status, BAR_PG, NPG)) break;
       // q, k rows normalised in place (k rows 0..63, q rows 64..127)
-      pipe_normalize<DVS>(t3, 0, tid, a.l2norm, hmax);
-      pipe_normalize<DVS>(t3, 64, tid, a.l2norm, hmax);
+      normalize_rows<M::T3_ATOM>(t3, 0, tid, a.l2norm, hmax);
+      normalize_rows<M::T3_ATOM>(t3, 64, tid, a.l2norm, hmax);
       named_bar(BAR_PG, NPG);     // the factor block, for beta
       // beta v in place
       for (int i = tid; i < C * DVS / 8; i += NPG) {
@@ -583,46 +740,29 @@ __global__ void __launch_bounds__(NTP, 1)
 
       // ---- L (quarters 0, 1; in X's place, plus FP32 diagonal blocks) and A (quarters 2, 3)
       const uint32_t Xb = pb + 128 * 128, Xwb = pb + 64 * 128;
-      {
+      // Q' = diag(e^{G_t}) Q in place, 128 threads j (MMA-a has finished
+      // reading Q); the two threads of a row walk their atoms half a row
+      // apart, so four rows' eight chunks fall on distinct bank groups
+      auto q_prime = [&](int j) {
+        const int row = j >> 1, c0 = (j & 1) * 64;
+        const float e = eg[row];
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 8) {
+          const int col = c0 + ((cc + 32 * (j & 1)) & 63);
+          scale_chunk_h(t3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(64 + row, col & 63), e);
+        }
+      };
+      if (!XPRE || quarter >= 2) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem + lane_off + PP + colhalf * 32, r);
         tc_wait_ld();
-        const int s0 = colhalf * 32;
-        float v[32];
         if (quarter < 2) {
-          const int t = quarter * 32 + lane;
-          const float bt = be[t], gm = g2m1[t];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int s2 = s0 + i;
-            v[i] = (s2 < t) ? bt * ex2(fminf(gm - g2[s2], 0.0f)) * __uint_as_float(r[i]) : 0.0f;
-          }
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            st_chunk_hc(Xb + swz(t, s0 + 8 * cc), &v[8 * cc], hmax);
-            // Xw's row starts zero: the inverse writes only its lower blocks,
-            // and the rows held K' for the chunk two back
-            st_s128(Xwb + swz(t, s0 + 8 * cc), 0u, 0u, 0u, 0u);
-          }
-          const int blk = t >> 4;
-          if ((blk >> 1) == colhalf) {
-            // the diagonal block's 16 columns are the first or second half of these 32
-            const uint32_t dst = sb + M::LD32 + (uint32_t)(blk * 256 + (t & 15) * 16) * 4;
-            if (blk & 1) {
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc)
-                st_s128(dst + cc * 16, __float_as_uint(v[16 + 4 * cc]), __float_as_uint(v[17 + 4 * cc]),
-                        __float_as_uint(v[18 + 4 * cc]), __float_as_uint(v[19 + 4 * cc]));
-            } else {
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc)
-                st_s128(dst + cc * 16, __float_as_uint(v[4 * cc]), __float_as_uint(v[1 + 4 * cc]),
-                        __float_as_uint(v[2 + 4 * cc]), __float_as_uint(v[3 + 4 * cc]));
-            }
-          }
+          build_l_row(r, quarter * 32 + lane, colhalf, Xb, Xwb, sb + M::LD32, be, g2m1, g2, hmax);
         } else {
           const int t = (quarter - 2) * 32 + lane;
           const float gt = g2[t];
+          const int s0 = colhalf * 32;
+          float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int s2 = s0 + i;
@@ -631,112 +771,18 @@ __global__ void __launch_bounds__(NTP, 1)
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) st_chunk_hc(pb + swz(t, s0 + 8 * cc), &v[8 * cc], hmax);
         }
-      }
-      named_bar(BAR_PG, NPG);
-
-      if (warp < 4) {
-        // ---- X = (I + L)^{-1} and Xw = X diag(beta_s e^{G_{s-1}}) (warps 0-3)
-        const float* d1 = fb + Fac::D1;
-        {
-          // every lane solves column j = lane % 16 (the two half-warps the
-          // same column): lanes 0-15 store X, lanes 16-31 store Xw
-          const int base = 16 * warp;
-          const int j = lane & 15;
-          const bool wside = lane >= 16;
-          const float4* lb4 = reinterpret_cast<const float4*>(smem + M::LD32 + warp * 1024);
-          float acc[16];
-#pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            float l[16];
-#pragma unroll
-            for (int cc = 0; cc < (t + 3) / 4; ++cc) {
-              const float4 v4 = lb4[t * 4 + cc];
-              l[4 * cc] = v4.x; l[4 * cc + 1] = v4.y; l[4 * cc + 2] = v4.z; l[4 * cc + 3] = v4.w;
-            }
-            float p0 = (t == j) ? 1.0f : 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
-#pragma unroll
-            for (int s2 = 0; s2 < t; ++s2) {
-              if ((s2 & 3) == 0) p0 = fmaf(-l[s2], acc[s2], p0);
-              if ((s2 & 3) == 1) p1 = fmaf(-l[s2], acc[s2], p1);
-              if ((s2 & 3) == 2) p2 = fmaf(-l[s2], acc[s2], p2);
-              if ((s2 & 3) == 3) p3 = fmaf(-l[s2], acc[s2], p3);
-            }
-            acc[t] = (t < j) ? 0.0f : (p0 + p1) + (p2 + p3);
-          }
-          const float dj = wside ? d1[base + j] : 1.0f;
-          const uint32_t dst = wside ? Xwb : Xb;
-          __syncwarp();
-          float am = 0.0f;
-#pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const float x = acc[t] * dj;
-            am = fmaxf(am, fabsf(x));
-            const __half hx = __float2half_rn(x);
-            asm volatile("st.shared.b16 [%0], %1;" ::"r"(dst + swz(base + t, base + j)), "h"(__half_as_ushort(hx))
-                         : "memory");
-          }
-          hmax = fmaxf(hmax, am);
-        }
-        named_bar(BAR_INV, 128);
-        uint32_t Pk[3][4];
-        const int g = lane >> 2, c4 = lane & 3;
-        {
-          uint32_t af[4];
-          frag_a(af, Xb, 16 * warp, 16 * warp, lane);
-#pragma unroll
-          for (int dd = 1; dd <= 3; ++dd) {
-            if (dd <= warp) {
-              float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};
-              uint32_t bf[4];
-              frag_b_kn(bf, Xb, 16 * warp, 16 * (warp - dd), lane);   // still L_ik
-              mma16816(p0, af, bf[0], bf[1]);
-              mma16816(p1, af, bf[2], bf[3]);
-              c_to_a(Pk[dd - 1], p0, p1);
-            }
-          }
-        }
-        __syncwarp();
-#pragma unroll
-        for (int d = 1; d < 4; ++d) {
-          if (warp >= d) {
-            const int i = warp, jb = warp - d;
-            float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int dd = 1; dd <= 3; ++dd) {
-              if (dd <= d) {
-                uint32_t bf[4];
-                frag_b_kn(bf, Xb, 16 * (i - dd), 16 * jb, lane);
-                mma16816(z0, Pk[dd - 1], bf[0], bf[1]);
-                mma16816(z1, Pk[dd - 1], bf[2], bf[3]);
-              }
-            }
-            const int r0 = 16 * i + g, cc = 16 * jb + 2 * c4;
-            const float da = d1[cc], db = d1[cc + 1], dc = d1[cc + 8], dd2 = d1[cc + 9];
-            hmax = fmaxf(hmax, fmaxf(fmaxf(fmaxf(fabsf(z0[0]), fabsf(z0[1])), fmaxf(fabsf(z0[2]), fabsf(z0[3]))),
-                                     fmaxf(fmaxf(fabsf(z1[0]), fabsf(z1[1])), fmaxf(fabsf(z1[2]), fabsf(z1[3])))));
-            st_s32(Xb + swz(r0, cc), pack_h2(-z0[0], -z0[1]));
-            st_s32(Xb + swz(r0 + 8, cc), pack_h2(-z0[2], -z0[3]));
-            st_s32(Xb + swz(r0, cc + 8), pack_h2(-z1[0], -z1[1]));
-            st_s32(Xb + swz(r0 + 8, cc + 8), pack_h2(-z1[2], -z1[3]));
-            st_s32(Xwb + swz(r0, cc), pack_h2(-z0[0] * da, -z0[1] * db));
-            st_s32(Xwb + swz(r0 + 8, cc), pack_h2(-z0[2] * da, -z0[3] * db));
-            st_s32(Xwb + swz(r0, cc + 8), pack_h2(-z1[0] * dc, -z1[1] * dd2));
-            st_s32(Xwb + swz(r0 + 8, cc + 8), pack_h2(-z1[2] * dc, -z1[3] * dd2));
-          }
-          named_bar(BAR_INV, 128);
-        }
       } else {
-        // ---- beside the inverse: Q' = diag(e^{G_t}) Q in place (warps 4-7;
-        // MMA-a has finished reading Q)
-        // (the two threads of a row walk their atoms half a row apart, so
-        // four rows' eight chunks fall on distinct bank groups)
-        const int j = tid - 128;
-        const int row = j >> 1, c0 = (j & 1) * 64;
-        const float e = eg[row];
-#pragma unroll
-        for (int cc = 0; cc < 64; cc += 8) {
-          const int col = c0 + ((cc + 32 * (j & 1)) & 63);
-          scale_chunk_h(t3 + (uint32_t)(col >> 6) * M::T3_ATOM + swz(64 + row, col & 63), e);
+        // X and Xw came with the chunk's loads: quarters 0, 1 take Q' beside A
+        q_prime((((warp >> 2) << 1) | (warp & 1)) * 32 + lane);
+      }
+      if (!XPRE) {
+        named_bar(BAR_PG, NPG);
+        if (warp < 4) {
+          // ---- X = (I + L)^{-1} and Xw = X diag(beta_s e^{G_{s-1}}) (warps 0-3)
+          chunk_inverse(reinterpret_cast<const float4*>(smem + M::LD32), Xb, Xwb, fb + Fac::D1, warp, lane, hmax,
+                        BAR_INV);
+        } else {
+          q_prime(tid - 128);   // beside the inverse (warps 4-7)
         }
       }
       fence_async_smem();
@@ -939,7 +985,7 @@ __global__ void __launch_bounds__(NTP, 1)
       tc_fence_after();
       // the beta-V tile of stage s is free: chunk c+2's v
       if (tid == LD_ISSUER && c + 2 < nchunks) {
-        pipe_load_v<DVS>(sb, &bar_ld[s], maps, a, b, h, dv_off, seg0 + t0 + 2 * C, s);
+        pipe_load_v<DVS, XPRE>(sb, &bar_ld[s], maps, a, b, h, dv_off, seg0 + t0 + 2 * C, s);
         if (s == 0) ++v0; else ++v1;
       }
       // ---- o rows (quarters 0, 1: token rows in lanes 0..63), 32 columns at a time
@@ -1042,9 +1088,9 @@ __global__ void __launch_bounds__(NTP, 1)
   // chunk loads still in flight after an early exit land before the CTA exits
   if (tid == LD_ISSUER) {
     // a stage whose k and q went out without its v: complete the phase
-    if (v0 < kq0) pipe_load_v<DVS>(sb, &bar_ld[0], maps, a, b, h, dv_off, seg0 + (int64_t)(2 * (kq0 - 1)) * C, 0);
+    if (v0 < kq0) pipe_load_v<DVS, XPRE>(sb, &bar_ld[0], maps, a, b, h, dv_off, seg0 + (int64_t)(2 * (kq0 - 1)) * C, 0);
     if (v1 < kq1)
-      pipe_load_v<DVS>(sb, &bar_ld[1], maps, a, b, h, dv_off, seg0 + (int64_t)(2 * (kq1 - 1) + 1) * C, 1);
+      pipe_load_v<DVS, XPRE>(sb, &bar_ld[1], maps, a, b, h, dv_off, seg0 + (int64_t)(2 * (kq1 - 1) + 1) * C, 1);
     for (int k = consumed[0]; k < kq0; ++k) mbar_wait(&bar_ld[0], (uint32_t)k & 1u, a.status);
     for (int k = consumed[1]; k < kq1; ++k) mbar_wait(&bar_ld[1], (uint32_t)k & 1u, a.status);
   }
@@ -1052,6 +1098,171 @@ __global__ void __launch_bounds__(NTP, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ===========================================================================
+// Inverse pre-pass: X and Xw of every chunk of every (batch, head) chain,
+// ahead of the scan.
+//
+// Nothing in X = (I + L)^{-1} or Xw = X diag(beta_s e^{G_{s-1}}) depends on
+// the state: L is built from the chunk's normalised keys and its gates alone.
+// So one wide pass computes them for all chunks at once, with every SM busy
+// and several CTAs per SM hiding one another's latency, and writes each
+// chunk's pair as the 16 KB shared-memory image that the scan's MMA-b reads
+// ([Xw; X]: 128 rows of 64 FP16, 128-byte swizzled).  The scan (XPRE) then
+// loads the image with one bulk copy beside the chunk's v instead of building
+// L and inverting on its critical path.  The arithmetic is the scan's own
+// (the same normalisation, K K^T on the same tensor-core MMA, the same L rows
+// and inverse), so the image holds the values the scan would compute.
+//
+// One CTA of four warps walks chunk-heads idx = (b * nch_T + chunk) * H + h:
+// TMA load of the chunk's 64 k rows, normalisation in place, K K^T into TMEM
+// by one tcgen05 MMA group (M = 128: the A operand's rows 64..127 are
+// whatever follows the k tile in shared memory; their products land in TMEM
+// lanes that are never read), the L rows (warps 0, 1: lanes 0..63), the
+// inverse (warps 0-3), the image to global memory.  The next chunk's k is
+// loaded as soon as the MMA has read this one.
+constexpr int NTI = 128;
+struct IMap {
+  static constexpr uint32_t KT = 0;                  // k: two 64-column atoms of 64 rows
+  static constexpr uint32_t K_ATOM = 64 * 128;
+  static constexpr uint32_t IMG = 2 * K_ATOM;        // [Xw; X]
+  static constexpr uint32_t LD32 = IMG + kImgBytes;  // FP32 diagonal blocks of L
+  static constexpr uint32_t F = LD32 + 4 * 16 * 16 * 4;
+  static constexpr uint32_t MISC = F + (Fac::BYTES + 15) / 16 * 16;
+  static constexpr uint32_t BYTES = MISC + 64;
+};
+static_assert(IMap::IMG % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+
+__global__ void __launch_bounds__(NTI, 6) chunk_inverse_kernel(const __grid_constant__ Args a,
+                                                            const __grid_constant__ Maps maps, uint8_t* img,
+                                                            int64_t B) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sb - sraw);
+  uint64_t* bar_ld = reinterpret_cast<uint64_t*>(smem + IMap::MISC);
+  uint64_t* bar_mma = bar_ld + 1;
+  uint64_t* bar_fin = bar_ld + 2;
+  uint32_t* tmem_ptr = reinterpret_cast<uint32_t*>(smem + IMap::MISC + 24);
+  float* fb = reinterpret_cast<float*>(smem + IMap::F);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t nch = a.nch_T, total = B * nch * a.H;
+  const uint32_t kt = sb + IMap::KT, Xwb = sb + IMap::IMG, Xb = Xwb + 64 * 128;
+  if (tid == 0) {
+    mbar_init(bar_ld, 1);
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_fin, 1);
+    fence_mbar_init();
+    prefetch_tmap(&maps.k);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_ptr, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr;
+  // tid 0: the k rows of chunk-head idx
+  auto load = [&](int64_t idx) {
+    const int h = (int)(idx % a.H);
+    const int64_t g = (idx / a.H) % nch;
+    const int b = (int)(idx / (a.H * nch));
+    mbar_arrive_expect_tx(bar_ld, 2 * IMap::K_ATOM);
+#pragma unroll
+    for (int at = 0; at < 2; ++at)
+      tma_load_3d(kt + at * IMap::K_ATOM, &maps.k, smem_u32(bar_ld), h * DK + 64 * at, (int32_t)(g * C), b);
+  };
+  int issued = 0, landed = 0;   // tid 0: k loads issued / waited for
+  if (tid == 0 && (int64_t)blockIdx.x < total) {
+    load(blockIdx.x);
+    issued = 1;
+  }
+  float hmax = 0.0f;
+  uint32_t it = 0;
+  // warp 3: the raw gates of chunk-head idx (zero past the end of the
+  // sequence), fetched one chunk-head ahead
+  float nla[2] = {0.f, 0.f}, nbs[2] = {0.f, 0.f};
+  auto fetch = [&](int64_t idx) {
+    const int h = (int)(idx % a.H);
+    const int64_t g = (idx / a.H) % nch;
+    const int b = (int)(idx / (a.H * nch));
+    fetch_gates(a, (int64_t)b * a.T, h, g * C, a.T, lane, nla, nbs);
+  };
+  if (warp == 3 && (int64_t)blockIdx.x < total) fetch(blockIdx.x);
+#pragma unroll 1
+  for (int64_t idx = blockIdx.x; idx < total; idx += gridDim.x, ++it) {
+    if (warp == 3) {
+      // the chunk's gate factors
+      const float la[2] = {nla[0], nla[1]}, bs[2] = {nbs[0], nbs[1]};
+      if (idx + gridDim.x < total) fetch(idx + gridDim.x);
+      fb[Fac::BE + 2 * lane] = bs[0];
+      fb[Fac::BE + 2 * lane + 1] = bs[1];
+      scan_gates(fb, la, bs, lane);
+    }
+    bool bad = !mbar_wait(bar_ld, it & 1u, a.status);
+    if (__syncthreads_or(bad)) break;
+    if (tid == 0) landed = issued;
+    normalize_rows<IMap::K_ATOM>(kt, 0, tid, a.l2norm, hmax);
+    normalize_rows<IMap::K_ATOM>(kt, 32, tid, a.l2norm, hmax);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // K K^T -> TMEM (lanes 0..63, 64 columns)
+    if (warp == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
+#pragma unroll
+      for (int j = 0; j < DK / 16; ++j) {
+        const uint64_t d = sdesc(kt + (j >> 2) * IMap::K_ATOM + (j & 3) * 32, 16);
+        mma_f16_warp(tmem, d, d, id, j > 0 ? 1u : 0u);
+      }
+      tc_commit_warp(bar_mma);
+    }
+    bad = !mbar_wait(bar_mma, it & 1u, a.status);
+    if (__syncthreads_or(bad)) break;
+    tc_fence_after();
+    // the k tile is free: the next chunk-head's k
+    if (tid == 0 && idx + gridDim.x < total) {
+      load(idx + gridDim.x);
+      ++issued;
+    }
+    if (warp < 2) {
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + ch * 32, r);
+        tc_wait_ld();
+        build_l_row(r, warp * 32 + lane, ch, Xb, Xwb, sb + IMap::LD32, fb + Fac::BE, fb + Fac::G2M1, fb + Fac::G2,
+                    hmax);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    chunk_inverse(reinterpret_cast<const float4*>(smem + IMap::LD32), Xb, Xwb, fb + Fac::D1, warp, lane, hmax, 1);
+    // the image out (the inverse ends at a barrier of all four warps)
+    uint4* dst = reinterpret_cast<uint4*>(img + idx * (int64_t)kImgBytes);
+#pragma unroll
+    for (int i = tid; i < (int)(kImgBytes / 16); i += NTI) dst[i] = ld_s128(Xwb + (uint32_t)i * 16);
+  }
+  // after an early exit: a k load still in flight lands before the CTA exits
+  if (tid == 0 && issued > landed)
+    for (uint32_t i = 0; i < kWaitLimit && !mbar_try_wait(bar_ld, (uint32_t)landed & 1u); ++i) __nanosleep(32);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) hmax = fmaxf(hmax, __shfl_xor_sync(0xffffffffu, hmax, o));
+  if (lane == 0 && hmax >= kHalfOverflow) report_status(a.status, GDN_ERR_RANGE);
+  // every MMA this CTA issued has completed before TMEM is freed
+  if (warp == 0) {
+    tc_commit_warp(bar_fin);
+    mbar_wait(bar_fin, 0, a.status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 
@@ -1071,19 +1282,49 @@ bool make_map_3d(CUtensorMap* map, const void* base, int64_t features, int64_t T
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DVS, bool O_F32>
+template <int DVS, bool O_F32, bool XPRE>
 int launch_dvs(const Args& a, const Maps& m, int64_t units, cudaStream_t stream) {
   const size_t smem = PMap<DVS>::BYTES + 1024;
-  cudaError_t e =
-      cudaFuncSetAttribute(delta_rule_pipe_kernel<DVS, O_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(delta_rule_pipe_kernel<DVS, O_F32, XPRE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return record_cuda_error(e);
-  delta_rule_pipe_kernel<DVS, O_F32><<<(unsigned)(units * a.nsplit), NTP, smem, stream>>>(a, m);
+  delta_rule_pipe_kernel<DVS, O_F32, XPRE><<<(unsigned)(units * a.nsplit), NTP, smem, stream>>>(a, m);
   return check_launch();
 }
 
+// XPRE (the precomputed inverse) runs with 128-column slices only: the
+// segmented path, the one that uses it.
 int launch_args(const Args& a, const Maps& m, int64_t units, int dvs, bool f32, cudaStream_t stream) {
-  if (dvs == 128) return f32 ? launch_dvs<128, true>(a, m, units, stream) : launch_dvs<128, false>(a, m, units, stream);
-  return f32 ? launch_dvs<64, true>(a, m, units, stream) : launch_dvs<64, false>(a, m, units, stream);
+  if (a.xinv) {
+    if (dvs != 128) return GDN_ERR_UNSUPPORTED_SHAPE;
+    return f32 ? launch_dvs<128, true, true>(a, m, units, stream) : launch_dvs<128, false, true>(a, m, units, stream);
+  }
+  if (dvs == 128)
+    return f32 ? launch_dvs<128, true, false>(a, m, units, stream) : launch_dvs<128, false, false>(a, m, units, stream);
+  return f32 ? launch_dvs<64, true, false>(a, m, units, stream) : launch_dvs<64, false, false>(a, m, units, stream);
+}
+
+// The pre-pass asks for the largest shared-memory carveout: with the default
+// the driver may size the SM's shared memory for one 40 KB CTA and leave the
+// rest to L1, while the pass needs several CTAs per SM to hide its latency.
+cudaError_t inverse_attributes(int smem) {
+  cudaError_t e = cudaFuncSetAttribute(chunk_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(chunk_inverse_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
+}
+
+int launch_inverse(const Args& a, const Maps& m, uint8_t* img, int64_t B, cudaStream_t stream) {
+  const int64_t total = B * a.nch_T * a.H;
+  if (total == 0) return GDN_OK;
+  const int smem = (int)IMap::BYTES + 1024;
+  cudaError_t e = inverse_attributes(smem);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  // one CTA per chunk-head (as many resident per SM as fit: 80 registers,
+  // 40 KB of shared memory); measured faster than a persistent grid sized
+  // by the occupancy query
+  chunk_inverse_kernel<<<(unsigned)total, NTI, smem, stream>>>(a, m, img, B);
+  return check_launch();
 }
 
 // ---------------------------------------------------------------------------
@@ -1106,45 +1347,83 @@ int launch_args(const Args& a, const Maps& m, int64_t units, int dvs, bool f32, 
 
 // E[b, p, h] = S_p for p = 0 .. nseg-1, S_0 = S0 (or 0), S_{p+1} = M_p S_p +
 // B_p with [M_p | B_p] = MB[b, p, h] ([d_k, d_k + dv]).  One CTA of 256
-// threads per (batch, head, 16 state columns): thread t owns row t/2 and
-// eight columns; the sixteen columns of S_p stay in shared memory.
+// threads per (batch, head, 16 state columns): thread t owns column t % 16 of
+// rows t / 16 + 16 i (i < 8); S_p's sixteen columns stay in shared memory, and
+// M_p is staged there by cp.async, double-buffered (M_{p+1} loads while
+// M_p S_p is formed), rows padded to 132 floats so that the two rows a warp
+// reads fall on distinct banks.  Each element sums B_p then k = 0 .. d_k-1 in
+// order.
+constexpr int CMB_LD = DK + 4;
+constexpr size_t CMB_SMEM = (size_t)(2 * DK * CMB_LD + DK * 16) * 4;
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 __global__ void __launch_bounds__(256) segment_combine_kernel(const float* __restrict__ MB,
                                                               const float* __restrict__ S0, float* __restrict__ E,
                                                               int H, int dv, int nseg) {
-  __shared__ float Ss[DK][16];
+  extern __shared__ float cmb[];
+  float* Mb = cmb;                      // [2][DK][CMB_LD]
+  float* Ss = cmb + 2 * DK * CMB_LD;    // [DK][16]
   const int ncb = dv / 16;
   const int cb = blockIdx.x % ncb, bh = blockIdx.x / ncb;
   const int b = bh / H, h = bh % H;
-  const int tid = threadIdx.x, r = tid >> 1, c0 = (tid & 1) * 8;
-  const int col = cb * 16 + c0;
+  const int tid = threadIdx.x, c = tid & 15, rg = tid >> 4;
+  const int col = cb * 16 + c;
   const int ld = DK + dv;
+  auto mb = [&](int p) { return MB + (((int64_t)b * (nseg - 1) + p) * H + h) * DK * ld; };
+  auto stage = [&](int p) {
+    const float* src = mb(p);
+    float* dst = Mb + (p & 1) * DK * CMB_LD;
+    for (int i = tid; i < DK * DK / 4; i += 256) {
+      const int r = i >> 5, k4 = (i & 31) * 4;
+      cp_async16(dst + r * CMB_LD + k4, src + (int64_t)r * ld + k4);
+    }
+    cp_async_commit();
+  };
+  if (nseg > 1) stage(0);
   float st[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) st[e] = S0 ? S0[(((int64_t)b * H + h) * DK + r) * dv + col + e] : 0.0f;
+  for (int i = 0; i < 8; ++i) st[i] = S0 ? S0[(((int64_t)b * H + h) * DK + rg + 16 * i) * dv + col] : 0.0f;
   for (int p = 0;; ++p) {
-    float* dst = E + ((((int64_t)b * nseg + p) * H + h) * DK + r) * dv + col;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = st[e];
+    for (int i = 0; i < 8; ++i) E[((((int64_t)b * nseg + p) * H + h) * DK + rg + 16 * i) * dv + col] = st[i];
     if (p + 1 == nseg) break;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) Ss[r][c0 + e] = st[e];
-    __syncthreads();
-    const float* mrow = MB + ((((int64_t)b * (nseg - 1) + p) * H + h) * DK + r) * ld;
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = mrow[DK + col + e];
-#pragma unroll 4
-    for (int k = 0; k < DK; k += 4) {
-      const float4 m4 = *reinterpret_cast<const float4*>(mrow + k);
-      const float mk[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(mk[kk], Ss[k + kk][c0 + e], acc[e]);
+    for (int i = 0; i < 8; ++i) Ss[(rg + 16 * i) * 16 + c] = st[i];
+    if (p + 2 < nseg) {
+      stage(p + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const float* M = Mb + (p & 1) * DK * CMB_LD;
+    const float* Bp = mb(p) + DK + col;
+    float acc[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) st[e] = acc[e];
+    for (int i = 0; i < 8; ++i) acc[i] = Bp[(int64_t)(rg + 16 * i) * ld];
+#pragma unroll 2
+    for (int k = 0; k < DK; k += 4) {
+      float s4[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) s4[kk] = Ss[(k + kk) * 16 + c];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 m = *reinterpret_cast<const float4*>(M + (rg + 16 * i) * CMB_LD + k);
+        acc[i] = fmaf(m.x, s4[0], acc[i]);
+        acc[i] = fmaf(m.y, s4[1], acc[i]);
+        acc[i] = fmaf(m.z, s4[2], acc[i]);
+        acc[i] = fmaf(m.w, s4[3], acc[i]);
+      }
+    }
+    __syncthreads();   // Ss and this M buffer are rewritten next
+#pragma unroll
+    for (int i = 0; i < 8; ++i) st[i] = acc[i];
   }
 }
 
@@ -1188,11 +1467,23 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool delta_rule_tc_supported(int dk, int dv, int64_t T) { return dk == DK && dv % 64 == 0 && T < ((int64_t)1 << 31); }
 
+namespace {
+// Workspace of the segmented path: [M_p | B_p] and the entry states, then the
+// [Xw; X] image of every chunk (the inverse pre-pass).  Both passes of the
+// segmented path walk every chunk, so the pre-pass saves one of the two
+// inversions of each chunk; in one piece per sequence the scan inverts each
+// chunk once, beside the state update, and a pre-pass would cost more than it
+// takes off the critical path (measured at B = 4, T = 8192, H = 32).
+size_t seg_bytes(int64_t B, int H, int dv, int P) {
+  return P > 1 ? align256(align256(seg_bytes_mb(B, H, dv, P)) + seg_bytes_e(B, H, dv, P)) : 0;
+}
+size_t img_bytes(int64_t B, int64_t T, int H) { return (size_t)(B * ((T + C - 1) / C) * H) * kImgBytes; }
+}  // namespace
+
 size_t delta_rule_tc_workspace(int64_t B, int64_t T, int H, int dk, int dv) {
-  if (!delta_rule_tc_supported(dk, dv, T)) return 0;
+  if (!delta_rule_tc_supported(dk, dv, T) || T <= 0) return 0;
   const SegPlan pl = plan_segments(B, T, H, dv, num_sms());
-  if (pl.P < 2) return 0;
-  return align256(seg_bytes_mb(B, H, dv, pl.P)) + seg_bytes_e(B, H, dv, pl.P);
+  return pl.P > 1 ? seg_bytes(B, H, dv, pl.P) + img_bytes(B, T, H) : 0;
 }
 
 int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t ld_q, int64_t ld_k,
@@ -1235,8 +1526,18 @@ int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v
     a.oq_g_out = oq->g_out;
   }
   const SegPlan pl = plan_segments(B, T, H, dv, sms);
-  const size_t need = pl.P > 1 ? align256(seg_bytes_mb(B, H, dv, pl.P)) + seg_bytes_e(B, H, dv, pl.P) : 0;
-  if (pl.P > 1 && ws && ws_bytes >= need && aligned(ws, 256)) {
+  const size_t need_seg = seg_bytes(B, H, dv, pl.P);
+  const bool ws_ok = ws && aligned(ws, 256);
+  // the inverse pre-pass, when the sequences are cut into segments and the
+  // workspace holds every chunk's image
+  if (pl.P > 1 && ws_ok && ws_bytes >= need_seg + img_bytes(B, T, H)) {
+    a.nch_T = (T + C - 1) / C;
+    uint8_t* img = static_cast<uint8_t*>(ws) + need_seg;
+    a.xinv = img;
+    const int st = launch_inverse(a, m, img, B, stream);
+    if (st) return st;
+  }
+  if (pl.P > 1 && ws_ok && ws_bytes >= need_seg) {
     float* MB = static_cast<float*>(ws);
     float* E = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(seg_bytes_mb(B, H, dv, pl.P)));
     // phase A: segments 0 .. P-2 from [I | 0]; the state transition and the
@@ -1255,7 +1556,10 @@ int launch_delta_rule_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v
     int st = launch_args(pa, m, B * (pl.P - 1) * H, 128, f32, stream);
     if (st) return st;
     // phase B: the entry state of every segment
-    segment_combine_kernel<<<(unsigned)(B * H * (dv / 16)), 256, 0, stream>>>(MB, S0, E, H, dv, pl.P);
+    cudaError_t ce =
+        cudaFuncSetAttribute(segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CMB_SMEM);
+    if (ce != cudaSuccess) return record_cuda_error(ce);
+    segment_combine_kernel<<<(unsigned)(B * H * (dv / 16)), 256, CMB_SMEM, stream>>>(MB, S0, E, H, dv, pl.P);
     st = check_launch();
     if (st) return st;
     // phase C: every segment from its entry state

@@ -170,3 +170,27 @@ def test_segmented_scan_equals_unsegmented_within_tolerance():
     o2, S2 = _lib.gdn_delta_rule_fwd(*args, S0=f32_cuda(S0), o_fp32=True, use_workspace=False)
     _lib.stream_check()
     assert rel_fro(to_np(o1), to_np(o2)) < TOL and rel_fro(to_np(S1), to_np(S2)) < TOL
+
+
+@pytest.mark.parametrize("B,T,H,o_fp32", [(1, 4100, 1, True), (1, 6000, 2, False)], ids=["fp32_o", "bf16_o"])
+def test_precomputed_inverse_is_bit_identical(B, T, H, o_fp32):
+    """Segmented sequences: with the full workspace a wide pre-pass computes
+    every chunk's (I + L)^{-1} and its beta-weighted copy once, with the
+    scan's own arithmetic (normalisation, tensor-core K K^T, L rows,
+    inverse), and both passes over the segments load them; a workspace short
+    of those 16 KB per chunk and head makes each pass invert on its own.
+    Both must give the same bits."""
+    q, k, v, la, be, S0 = _case(B, T, H, 128, 128, 91 + T, with_s0=True)
+    args = (bf16_cuda(q), bf16_cuda(k), bf16_cuda(v), f32_cuda(la), f32_cuda(be))
+    full = int(_lib.lib().gdn_delta_rule_workspace_size(B, T, H, 128, 128))
+    img = B * ((T + 63) // 64) * H * 16384
+    assert full > img
+    o1, S1 = _lib.gdn_delta_rule_fwd(*args, S0=f32_cuda(S0), o_fp32=o_fp32, workspace_bytes=full)
+    o2, S2 = _lib.gdn_delta_rule_fwd(*args, S0=f32_cuda(S0), o_fp32=o_fp32, workspace_bytes=full - img)
+    _lib.stream_check()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    o_ref, S_ref = delta_rule_chunked(q, k, v, la, be, S0=S0)
+    if not o_fp32:
+        from oracle.nvfp4 import round_bf16
+        o_ref = round_bf16(o_ref)
+    assert rel_fro(to_np(o1), o_ref) < (TOL if o_fp32 else 3e-3) and rel_fro(to_np(S1), S_ref) < TOL
