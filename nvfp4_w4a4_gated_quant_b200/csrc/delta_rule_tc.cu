@@ -1116,13 +1116,14 @@ __global__ void __launch_bounds__(NTP, 1)
 // (the same normalisation, K K^T on the same tensor-core MMA, the same L rows
 // and inverse), so the image holds the values the scan would compute.
 //
-// One CTA of four warps walks chunk-heads idx = (b * nch_T + chunk) * H + h:
-// TMA load of the chunk's 64 k rows, normalisation in place, K K^T into TMEM
-// by one tcgen05 MMA group (M = 128: the A operand's rows 64..127 are
-// whatever follows the k tile in shared memory; their products land in TMEM
-// lanes that are never read), the L rows (warps 0, 1: lanes 0..63), the
-// inverse (warps 0-3), the image to global memory.  The next chunk's k is
-// loaded as soon as the MMA has read this one.
+// One CTA of four warps per chunk-head idx = (b * nch_T + chunk) * H + h (the
+// launch gives each CTA one; the loop also walks a grid-stride range, loading
+// the next chunk's k as soon as the MMA has read this one): TMA load of the
+// chunk's 64 k rows, normalisation in place, K K^T into TMEM by one tcgen05
+// MMA group (M = 128: the A operand's rows 64..127 are whatever follows the k
+// tile in shared memory; their products land in TMEM lanes that are never
+// read), the L rows (warps 0, 1: lanes 0..63), the inverse (warps 0-3), the
+// image to global memory.
 constexpr int NTI = 128;
 struct IMap {
   static constexpr uint32_t KT = 0;                  // k: two 64-column atoms of 64 rows
