@@ -393,14 +393,16 @@ def _token_stride(t, name):
 
 
 def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=False, o=None, S_T=None,
-                       want_state=True, stream=None, mma_sync=False, use_workspace=True, workspace_bytes=None):
+                       want_state=True, stream=None, mma_sync=False, use_workspace=True, workspace_bytes=None,
+                       workspace=None):
     """q, k [B, T, H, dk], v [B, T, H, dv] bf16 (heads contiguous, token stride
     free); log_alpha, beta FP32 [B, T, H] contiguous; S0 FP32 [B, H, dk, dv].
     ``mma_sync`` selects the warp-level mma.sync kernel where the tcgen05 one
     would run; ``use_workspace=False`` passes no workspace (long sequences on
     few chains then run in one piece instead of segments, and each chunk's
     inverse is computed inside the scan); ``workspace_bytes`` passes a
-    workspace of that size instead of the queried one.
+    workspace of that size instead of the queried one; ``workspace`` (a uint8
+    tensor on the device) passes the caller's own.
     Returns (o [B, T, H, dv] bf16 or FP32, S_T FP32 or None)."""
     lds = []
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -429,6 +431,9 @@ def gdn_delta_rule_fwd(q, k, v, log_alpha, beta, S0=None, l2norm=True, o_fp32=Fa
     if workspace_bytes is not None:
         wsz = int(workspace_bytes)
     ws = torch.empty(wsz, dtype=torch.uint8, device=dev) if wsz else None
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+        ws, wsz = workspace, workspace.numel()
     check(L.gdn_delta_rule_fwd(_ptr(q), _ptr(k), _ptr(v), lds[0], lds[1], lds[2], _ptr(log_alpha),
                                _ptr(beta), _ptr(S0), B, T, H, dk, dv, flags, _ptr(o), _ptr(S_T), _ptr(ws), wsz,
                                _stream(stream)))

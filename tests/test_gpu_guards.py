@@ -122,6 +122,27 @@ def test_scan_stays_in_bounds_and_writes_everything(B, T, H, d, mma_sync, o_fp32
     assert rel_fro(to_np(S_t), S_ref) < 2e-3
 
 
+def test_segmented_scan_workspace_stays_in_bounds():
+    """Sequences cut into segments: the call writes the segment states and
+    every chunk's inverse image into the caller's workspace, and nothing past
+    either end of it; a second call on the same (now stale) workspace gives
+    the same bits."""
+    B, T, H, d = 1, 2000, 2, 128
+    wsz = int(_lib.lib().gdn_delta_rule_workspace_size(B, T, H, d, d))
+    assert wsz >= B * ((T + 63) // 64) * H * 16384
+    rng = np.random.default_rng(5)
+    q, k, v = (bf16_cuda(rng.standard_normal((B, T, H, d)).astype(np.float32)) for _ in range(3))
+    la = f32_cuda(-rng.uniform(0, 1, (B, T, H)).astype(np.float32))
+    be = f32_cuda(rng.uniform(0, 1, (B, T, H)).astype(np.float32))
+    ws = Guarded(wsz, torch.uint8, 0x5A)
+    o1, S1 = _lib.gdn_delta_rule_fwd(q, k, v, la, be, workspace=ws.t)
+    o2, S2 = _lib.gdn_delta_rule_fwd(q, k, v, la, be, workspace=ws.t)
+    _lib.stream_check()
+    assert ws.canaries_intact()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    assert _nan_free(o1) and _nan_free(S1)
+
+
 def test_decode_step_stays_in_bounds_and_writes_everything():
     B, T, H, d = 3, 5, 2, 128
     rng = np.random.default_rng(5)
