@@ -9,9 +9,9 @@
 //            first from a carried state, else zero)
 //   out    = o / sqrt(mean_dv(o^2) + 1e-6) * gamma * SiLU(g)   per (token, head)
 // Both are HBM-bound elementwise passes: FP32 arithmetic on bf16 storage,
-// 8- and 16-byte vectors with several rows in flight per thread, one thread
-// per four channels (convolution) or DV/8 lanes per (token, head) row
-// (norm).  SiLU(u) = u sigmoid(u) with
+// 16-byte vectors with several rows in flight per thread, one thread per
+// eight channels (convolution, its rows staged by cp.async) or DV/8 lanes per
+// (token, head) row (norm).  SiLU(u) = u sigmoid(u) with
 // sigmoid(u) = 1/2 + tanh(u/2)/2 on the SFU's tanh.approx (relative error
 // ~2^-11, below the bf16 rounding of the stored result), so the passes stay
 // memory-bound.
@@ -26,7 +26,8 @@ namespace {
 constexpr int CW = 4;          // kernel width
 constexpr int CONV_TOK = 64;   // tokens one thread walks
 constexpr int CONV_THREADS = 256;
-constexpr int CONV_NR = 4;     // input rows per group; two groups in flight
+constexpr int CONV_NR = 8;     // input rows per group; two groups staged
+constexpr size_t CONV_SMEM = (size_t)2 * CONV_NR * CONV_THREADS * 16;
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -48,93 +49,90 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
                     pack_bf16x2(f[6], f[7]));
 }
 
-__device__ __forceinline__ void unpack4(const uint2& u, float* f) {
-  f[0] = bf16_bits_to_f32(u.x & 0xFFFFu);
-  f[1] = bf16_bits_to_f32(u.x >> 16);
-  f[2] = bf16_bits_to_f32(u.y & 0xFFFFu);
-  f[3] = bf16_bits_to_f32(u.y >> 16);
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ uint2 pack4(const float* f) {
-  return make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// grid (channel quads / CONV_THREADS, token blocks, batch): a thread keeps
-// the three previous inputs of its four channels in registers while it walks
-// CONV_TOK tokens, reading each input row once, in groups of CONV_NR rows.
+// grid (channel octets / CONV_THREADS, token blocks, batch): a thread keeps
+// the three previous inputs of its eight channels in registers while it walks
+// CONV_TOK tokens, reading each input row once.  Its rows arrive by cp.async
+// (16 bytes each) into its own slots of a shared-memory stage, CONV_NR rows a
+// group, the next group in flight while this one is computed: the bytes in
+// flight sit in shared memory, not in registers.
 __global__ void __launch_bounds__(CONV_THREADS) short_conv_kernel(const uint16_t* __restrict__ x, int64_t T, int64_t C,
                                                                   int64_t ld_x, const float* __restrict__ w,
                                                                   const uint16_t* __restrict__ state_in,
                                                                   uint16_t* __restrict__ y, int64_t ld_y,
                                                                   uint16_t* __restrict__ state_out) {
+  extern __shared__ uint4 conv_stage[];   // [2][CONV_NR][CONV_THREADS]
   const int64_t cv = (int64_t)blockIdx.x * CONV_THREADS + threadIdx.x;
-  if (cv * 4 >= C) return;
-  const int64_t c0 = cv * 4;
+  if (cv * 8 >= C) return;
+  const int64_t c0 = cv * 8;
   const int64_t b = blockIdx.z;
   const int64_t t_begin = (int64_t)blockIdx.y * CONV_TOK;
   const int64_t t_end = t_begin + CONV_TOK < T ? t_begin + CONV_TOK : T;
-  float wk[4][CW];
+  auto slot = [&](int buf, int u) { return &conv_stage[(buf * CONV_NR + u) * CONV_THREADS + threadIdx.x]; };
+  // rows t .. t+n-1 into stage buf (one commit group)
+  auto issue = [&](int64_t t, int buf, int64_t n) {
+    for (int u = 0; u < n; ++u) cp_async16(slot(buf, u), x + (b * T + t + u) * ld_x + c0);
+    cp_async_commit();
+  };
+  issue(t_begin, 0, t_end - t_begin < CONV_NR ? t_end - t_begin : CONV_NR);
+  float wk[8][CW];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
+  for (int e = 0; e < 8; ++e) {
     const float4 w4 = *reinterpret_cast<const float4*>(w + (c0 + e) * CW);
     wk[e][0] = w4.x; wk[e][1] = w4.y; wk[e][2] = w4.z; wk[e][3] = w4.w;
   }
-  float win[3][4];
+  float win[3][8];
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
     const int64_t t = t_begin - 3 + i;
     if (t >= 0) {
-      unpack4(*reinterpret_cast<const uint2*>(x + (b * T + t) * ld_x + c0), win[i]);
+      unpack8(*reinterpret_cast<const uint4*>(x + (b * T + t) * ld_x + c0), win[i]);
     } else if (state_in) {
-      unpack4(*reinterpret_cast<const uint2*>(state_in + (b * 3 + (t + 3)) * C + c0), win[i]);
+      unpack8(*reinterpret_cast<const uint4*>(state_in + (b * 3 + (t + 3)) * C + c0), win[i]);
     } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) win[i][e] = 0.0f;
+      for (int e = 0; e < 8; ++e) win[i][e] = 0.0f;
     }
   }
-  auto step = [&](const uint2& raw, int64_t t) {
-    float cur[4], out[4];
-    unpack4(raw, cur);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float acc = wk[e][0] * win[0][e];
-      acc = fmaf(wk[e][1], win[1][e], acc);
-      acc = fmaf(wk[e][2], win[2][e], acc);
-      acc = fmaf(wk[e][3], cur[e], acc);
-      out[e] = silu_f(acc);
-      win[0][e] = win[1][e];
-      win[1][e] = win[2][e];
-      win[2][e] = cur[e];
+  int g = 0;
+  for (int64_t t = t_begin; t < t_end; t += CONV_NR, ++g) {
+    const int64_t n = t_end - t < CONV_NR ? t_end - t : CONV_NR;
+    if (t + CONV_NR < t_end) {
+      const int64_t rest = t_end - t - CONV_NR;
+      issue(t + CONV_NR, (g + 1) & 1, rest < CONV_NR ? rest : CONV_NR);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    *reinterpret_cast<uint2*>(y + (b * T + t) * ld_y + c0) = pack4(out);
-  };
-  // groups of CONV_NR rows: the next group's loads are issued before this
-  // group's arithmetic and stores
-  int64_t t = t_begin;
-  uint2 cur[CONV_NR], nxt[CONV_NR];
-  if (t + CONV_NR <= t_end) {
+    for (int u = 0; u < n; ++u) {
+      float cur[8], out[8];
+      unpack8(*slot(g & 1, u), cur);
 #pragma unroll
-    for (int u = 0; u < CONV_NR; ++u) cur[u] = *reinterpret_cast<const uint2*>(x + (b * T + t + u) * ld_x + c0);
-  }
-  for (; t + CONV_NR <= t_end; t += CONV_NR) {
-    const bool more = t + 2 * CONV_NR <= t_end;
-    if (more) {
-#pragma unroll
-      for (int u = 0; u < CONV_NR; ++u)
-        nxt[u] = *reinterpret_cast<const uint2*>(x + (b * T + t + CONV_NR + u) * ld_x + c0);
-    }
-#pragma unroll
-    for (int u = 0; u < CONV_NR; ++u) step(cur[u], t + u);
-    if (more) {
-#pragma unroll
-      for (int u = 0; u < CONV_NR; ++u) cur[u] = nxt[u];
+      for (int e = 0; e < 8; ++e) {
+        float acc = wk[e][0] * win[0][e];
+        acc = fmaf(wk[e][1], win[1][e], acc);
+        acc = fmaf(wk[e][2], win[2][e], acc);
+        acc = fmaf(wk[e][3], cur[e], acc);
+        out[e] = silu_f(acc);
+        win[0][e] = win[1][e];
+        win[1][e] = win[2][e];
+        win[2][e] = cur[e];
+      }
+      *reinterpret_cast<uint4*>(y + (b * T + t + u) * ld_y + c0) = pack8(out);
     }
   }
-  for (; t < t_end; ++t) step(*reinterpret_cast<const uint2*>(x + (b * T + t) * ld_x + c0), t);
   // the last three inputs (carried state included) for the next call
   if (state_out && t_end == T) {
 #pragma unroll
-    for (int i = 0; i < 3; ++i)
-      *reinterpret_cast<uint2*>(state_out + (b * 3 + i) * C + c0) = pack4(win[i]);
+    for (int i = 0; i < 3; ++i) *reinterpret_cast<uint4*>(state_out + (b * 3 + i) * C + c0) = pack8(win[i]);
   }
 }
 
@@ -217,9 +215,16 @@ int launch_short_conv(const uint16_t* x, int64_t B, int64_t T, int64_t C, int64_
                              : cudaMemsetAsync(state_out, 0, (size_t)B * 3 * C * 2, stream);
     return e == cudaSuccess ? GDN_OK : record_cuda_error(e);
   }
-  const int64_t vecs = C / 4;
+  const int64_t vecs = C / 8;
   dim3 grid((unsigned)cdiv(vecs, CONV_THREADS), (unsigned)cdiv(T, CONV_TOK), (unsigned)B);
-  short_conv_kernel<<<grid, CONV_THREADS, 0, stream>>>(x, T, C, ld_x, w, state_in, y, ld_y, state_out);
+  // 64 KB of stage per block: three blocks per SM (80 registers) need the
+  // largest shared-memory carveout, which the driver may not pick by itself
+  cudaError_t e = cudaFuncSetAttribute(short_conv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CONV_SMEM);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(short_conv_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  short_conv_kernel<<<grid, CONV_THREADS, CONV_SMEM, stream>>>(x, T, C, ld_x, w, state_in, y, ld_y, state_out);
   return check_launch();
 }
 
