@@ -295,8 +295,8 @@ int gdn_delta_rule_fwd(const void* q, const void* k, const void* v,
  * Step 4, token by token (decode): the recurrence itself, without chunking.
  *
  * Passage: as gdn_delta_rule_fwd ("Anthology of the SOTA, theory-128",
- * section "The account").  Each (batch, head) chain keeps its state in
- * registers across the T tokens of the call and walks them in order:
+ * section "The account").  Each (batch, head) chain keeps its state on chip
+ * (shared memory) across the T tokens of the call and walks them in order:
  *   r_t = S_{t-1}^T k_t     (alpha_t S_{t-1}^T k_t with GDN_DR_DECAYED_READ,
  *                            the reading S_t = alpha_t (I - beta_t k_t k_t^T)
  *                            S_{t-1} + beta_t k_t v_t^T),

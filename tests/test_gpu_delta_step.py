@@ -59,6 +59,30 @@ def test_step_matches_sequential_oracle(B, T, H, dk, dv, seed, decayed):
     assert rel_fro(o, o_ref) < TOL
 
 
+@pytest.mark.parametrize("dk,dv,decayed", [(128, 128, False), (64, 32, True)])
+def test_step_element_aligned_state(dk, dv, decayed):
+    """A state buffer aligned to its element but not to 16 bytes is copied
+    to and from shared memory in 4-byte pieces instead of 16-byte ones; the
+    arithmetic is the same, so the results are the same bits as for an
+    aligned state, and match the oracle."""
+    B, T, H = 2, 3, 3
+    q, k, v, la, be, S0 = _case(B, T, H, dk, dv, 11 + dk)
+    args = (bf16_cuda(q), bf16_cuda(k), bf16_cuda(v), f32_cuda(la), f32_cuda(be))
+    n = B * H * dk * dv
+    raw_in = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    raw_out = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    S_in = raw_in[1:].view(B, H, dk, dv)          # 4-byte aligned, not 16
+    S_in.copy_(f32_cuda(S0))
+    S_out = raw_out[1:].view(B, H, dk, dv)
+    o_e, _ = _lib.gdn_delta_rule_step(*args, S=S_in, S_out=S_out, o_fp32=True, decayed_read=decayed)
+    o_a, S_a = _lib.gdn_delta_rule_step(*args, S=f32_cuda(S0), o_fp32=True, decayed_read=decayed)
+    _lib.stream_check()
+    assert torch.equal(o_e, o_a) and torch.equal(S_out, S_a)
+    o_ref, S_ref = delta_rule_sequential(q, k, v, la, be, S0=S0, decayed_read=decayed)
+    assert rel_fro(to_np(S_a).astype(np.float64), S_ref) < TOL
+    assert rel_fro(to_np(o_a).astype(np.float64), o_ref) < TOL
+
+
 def test_step_bf16_output():
     q, k, v, la, be, S0 = _case(2, 3, 4, 128, 128, 5)
     o, _ = _step(q, k, v, la, be, S0, o_fp32=False)
