@@ -16,6 +16,7 @@ of the method) on the host cores over a bounded sample of the same workload.
 import argparse
 import json
 import os
+import shutil
 import statistics
 import subprocess
 import sys
@@ -59,16 +60,35 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.skip = 0
+
+    def _lines(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for _ in f)
+        except OSError:
+            return 0
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
+        cmd = ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+               "-lms", "20"]
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+            # line-buffered, so that every sample reaches the file at once
+            self.proc = subprocess.Popen((["stdbuf", "-oL"] if shutil.which("stdbuf") else []) + cmd,
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        # nvidia-smi takes a moment to start: wait for its first sample, so that
+        # the samples after it fall inside the timed region that follows
+        deadline = time.time() + 10
+        while self.proc is not None and self.proc.poll() is None and time.time() < deadline:
+            n = self._lines()
+            if n:
+                self.skip = n
+                break
+            time.sleep(0.005)
         return self
 
     def __exit__(self, *exc):
@@ -87,8 +107,11 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
             os.unlink(self.path)
+        inside = rows[self.skip:]   # the samples taken during the timed region
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        adjacent = not inside
+        rows = inside or rows[-1:]   # else the sample taken just before the region began
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         reasons = set()
@@ -98,8 +121,12 @@ class ClockSampler:
                 if val.lower().startswith("active"):
                     reasons.add(n)
         loaded = [s for s in sm if smax and s > 0.3 * max(smax)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons), "samples": len(rows)}
+        out = {"sm_mhz": statistics.median(loaded) if loaded else None,
+               "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+               "samples": len(inside)}
+        if adjacent:
+            out["note"] = "no sample inside the timed region; the one taken just before it"
+        return out
 
 
 # ---------------------------------------------------- multi-rank plumbing --
