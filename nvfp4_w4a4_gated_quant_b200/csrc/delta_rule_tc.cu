@@ -418,12 +418,12 @@ __device__ __forceinline__ void pipe_load_v(uint32_t sb, uint64_t* bar, const Ma
                 kImgBytes, bar_s);
 }
 
-// In place: the bf16 rows r0 .. r0+nthreads/4-1 of a tile of 64-column atoms
-// ATOM bytes apart -> L2-normalised FP16 (four threads per row, 32 columns
-// each).  Thread pq of a row takes the
-// 16-byte chunks pq and pq + 4 of both 64-column atoms, in an order that puts
-// the eight threads of two adjacent rows on eight distinct swizzled bank
-// groups (the plain column order hit every bank group twice).
+// In place: the bf16 rows r0 .. r0 + nthreads/4 - 1 of a tile of 64-column
+// atoms ATOM bytes apart -> L2-normalised FP16 (four threads per row, 32
+// columns each).  Thread pq of a row takes the 16-byte chunks pq and pq + 4
+// of both 64-column atoms, in an order that puts the eight threads of two
+// adjacent rows on eight distinct swizzled bank groups (the plain column
+// order hit every bank group twice).
 template <uint32_t ATOM>
 __device__ __forceinline__ void normalize_rows(uint32_t t3, int r0, int tid, int l2norm, float& hmax) {
   constexpr int QC = DK / 4;
@@ -1108,7 +1108,7 @@ __global__ void __launch_bounds__(NTP, 1)
 // Nothing in X = (I + L)^{-1} or Xw = X diag(beta_s e^{G_{s-1}}) depends on
 // the state: L is built from the chunk's normalised keys and its gates alone.
 // So one wide pass computes them for all chunks at once, with every SM busy
-// and several CTAs per SM hiding one another's latency, and writes each
+// and several CTAs per SM, and writes each
 // chunk's pair as the 16 KB shared-memory image that the scan's MMA-b reads
 // ([Xw; X]: 128 rows of 64 FP16, 128-byte swizzled).  The scan (XPRE) then
 // loads the image with one bulk copy beside the chunk's v instead of building
