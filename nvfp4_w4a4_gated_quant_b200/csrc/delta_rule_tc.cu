@@ -28,6 +28,7 @@
 // off-diagonal blocks level by level).
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -1324,7 +1325,9 @@ int launch_inverse(const Args& a, const Maps& m, uint8_t* img, int64_t B, cudaSt
   // one CTA per chunk-head (as many resident per SM as fit: 80 registers,
   // 40 KB of shared memory); measured faster than a persistent grid sized
   // by the occupancy query
-  chunk_inverse_kernel<<<(unsigned)total, NTI, smem, stream>>>(a, m, img, B);
+  // (the kernel walks a grid-stride range, so a grid capped below 2^31
+  // still covers any count)
+  chunk_inverse_kernel<<<(unsigned)std::min<int64_t>(total, (int64_t)1 << 30), NTI, smem, stream>>>(a, m, img, B);
   return check_launch();
 }
 
