@@ -143,6 +143,39 @@ def test_segmented_scan_workspace_stays_in_bounds():
     assert _nan_free(o1) and _nan_free(S1)
 
 
+@pytest.mark.parametrize("B,T,C", [(2, 150, 96), (1, 77, 6176), (3, 1, 40)], ids=["ragged", "layer_width", "one_token"])
+def test_short_conv_stays_in_bounds_and_writes_everything(B, T, C):
+    """The convolution's output and carried state: rows staged through shared
+    memory in groups of eight (ragged last group, a last token block shorter
+    than 64), nothing written outside either buffer, nothing left unwritten."""
+    from oracle.conv_norm import short_conv
+    rng = np.random.default_rng(B * T + C)
+    x = bf16_cuda(rng.standard_normal((B, T, C)).astype(np.float32))
+    w = f32_cuda(rng.uniform(-0.8, 0.8, (C, 4)).astype(np.float32))
+    st_in = bf16_cuda(rng.standard_normal((B, 3, C)).astype(np.float32))
+    y = Guarded(B * T * C, torch.bfloat16, float("nan"))
+    st = Guarded(B * 3 * C, torch.bfloat16, float("nan"))
+    _lib.gdn_short_conv(x, w, state_in=st_in, y=y.t.view(B, T, C), state_out=st.t.view(B, 3, C))
+    _lib.stream_check()
+    assert y.canaries_intact() and st.canaries_intact()
+    assert _nan_free(y.t) and _nan_free(st.t)
+    y_ref, st_ref = short_conv(to_np(x), to_np(w), state=to_np(st_in))
+    assert rel_fro(to_np(y.t).reshape(B, T, C), nvfp4.round_bf16(y_ref)) < 2e-3
+    np.testing.assert_array_equal(to_np(st.t).reshape(B, 3, C), st_ref)
+
+
+def test_gated_rmsnorm_stays_in_bounds_and_writes_everything():
+    M, H, dv = 333, 3, 128
+    rng = np.random.default_rng(7)
+    o = bf16_cuda(rng.standard_normal((M, H * dv)).astype(np.float32))
+    g = bf16_cuda(rng.standard_normal((M, H * dv)).astype(np.float32))
+    gamma = f32_cuda(rng.uniform(0.5, 1.5, dv).astype(np.float32))
+    y = Guarded(M * H * dv, torch.bfloat16, float("nan"))
+    _lib.gdn_gated_rmsnorm(o, g, gamma, H, y=y.t.view(M, H * dv))
+    _lib.stream_check()
+    assert y.canaries_intact() and _nan_free(y.t)
+
+
 def test_decode_step_stays_in_bounds_and_writes_everything():
     B, T, H, d = 3, 5, 2, 128
     rng = np.random.default_rng(5)
