@@ -1353,12 +1353,12 @@ int launch_inverse(const Args& a, const Maps& m, uint8_t* img, int64_t B, cudaSt
 // B_p with [M_p | B_p] = MB[b, p, h] ([d_k, d_k + dv]).  One CTA of 256
 // threads per (batch, head, 16 state columns): thread t owns column t % 16 of
 // rows t / 16 + 16 i (i < 8); S_p's sixteen columns stay in shared memory, and
-// M_p is staged there by cp.async, double-buffered (M_{p+1} loads while
-// M_p S_p is formed), rows padded to 132 floats so that the two rows a warp
-// reads fall on distinct banks.  Each element sums B_p then k = 0 .. d_k-1 in
-// order.
+// M_p with the CTA's 16 columns of B_p is staged there by cp.async,
+// double-buffered (p + 1's load while M_p S_p is formed), rows of M padded to
+// 132 floats so that the two rows a warp reads fall on distinct banks.  Each
+// element sums B_p then k = 0 .. d_k-1 in order.
 constexpr int CMB_LD = DK + 4;
-constexpr size_t CMB_SMEM = (size_t)(2 * DK * CMB_LD + DK * 16) * 4;
+constexpr size_t CMB_SMEM = (size_t)(2 * DK * CMB_LD + 2 * DK * 16 + DK * 16) * 4;
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
@@ -1372,7 +1372,8 @@ __global__ void __launch_bounds__(256) segment_combine_kernel(const float* __res
                                                               int H, int dv, int nseg) {
   extern __shared__ float cmb[];
   float* Mb = cmb;                      // [2][DK][CMB_LD]
-  float* Ss = cmb + 2 * DK * CMB_LD;    // [DK][16]
+  float* Bb = Mb + 2 * DK * CMB_LD;     // [2][DK][16]: this CTA's 16 columns of B_p
+  float* Ss = Bb + 2 * DK * 16;         // [DK][16]
   const int ncb = dv / 16;
   const int cb = blockIdx.x % ncb, bh = blockIdx.x / ncb;
   const int b = bh / H, h = bh % H;
@@ -1386,6 +1387,11 @@ __global__ void __launch_bounds__(256) segment_combine_kernel(const float* __res
     for (int i = tid; i < DK * DK / 4; i += 256) {
       const int r = i >> 5, k4 = (i & 31) * 4;
       cp_async16(dst + r * CMB_LD + k4, src + (int64_t)r * ld + k4);
+    }
+    float* bdst = Bb + (p & 1) * DK * 16;
+    for (int i = tid; i < DK * 4; i += 256) {
+      const int r = i >> 2, c4 = (i & 3) * 4;
+      cp_async16(bdst + r * 16 + c4, src + (int64_t)r * ld + DK + cb * 16 + c4);
     }
     cp_async_commit();
   };
@@ -1407,10 +1413,10 @@ __global__ void __launch_bounds__(256) segment_combine_kernel(const float* __res
     }
     __syncthreads();
     const float* M = Mb + (p & 1) * DK * CMB_LD;
-    const float* Bp = mb(p) + DK + col;
+    const float* Bp = Bb + (p & 1) * DK * 16;
     float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = Bp[(int64_t)(rg + 16 * i) * ld];
+    for (int i = 0; i < 8; ++i) acc[i] = Bp[(rg + 16 * i) * 16 + c];
 #pragma unroll 2
     for (int k = 0; k < DK; k += 4) {
       float s4[4];
