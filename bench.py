@@ -496,6 +496,7 @@ def standalone_kernels(args, torch, _lib, inputs, dev, stream, which=None):
         _lib.gemm_bf16(xc, xs, gx, wc, wsc, gw, M, N, K, out=y)
     e1.record(stream)
     torch.cuda.synchronize()
+    _lib.stream_check()   # a kernel that gave up (bounded waits) raises instead of timing
     ms = e0.elapsed_time(e1) / reps
     tf = 2.0 * M * N * K / (ms / 1e3) / 1e12
     ceil = fp4_ceiling_tflops(torch, _lib, stream)
@@ -538,6 +539,7 @@ def standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps):
             _lib.gdn_delta_rule_fwd(q, k, v, la, be, o=o, S_T=S, mma_sync=mma_sync)
         e1.record(stream)
         torch.cuda.synchronize()
+        _lib.stream_check()
         ms = e0.elapsed_time(e1) / reps
         gbs = nbytes / (ms / 1e3) / 1e9
         out[key] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
@@ -560,6 +562,7 @@ def standalone_scan(args, torch, _lib, dev, stream, out, pk, e0, e1, reps):
         _lib.gdn_delta_rule_step(q, k, v, la, be, S=S, S_out=S, o=o)
     e1.record(stream)
     torch.cuda.synchronize()
+    _lib.stream_check()
     ms = e0.elapsed_time(e1) / reps
     gbs = nbytes / (ms / 1e3) / 1e9
     out["decode_step_B64_H32_d128"] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1),
